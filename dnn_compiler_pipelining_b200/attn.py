@@ -1,0 +1,154 @@
+"""Thin ctypes binding of libattn_b200.so (C ABI in include/attn.h).
+
+Argument marshalling only: every step of the attention forward runs in the
+library's CUDA kernels.  PyTorch supplies device memory and streams.  There is
+no fallback: if the library is missing or the device is not an sm_100 GPU,
+calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libattn_b200.so")
+
+ATTN_OK = 0
+ATTN_ERR_DEVICE_TIMEOUT = 6
+STATUS_NAMES = {0: "ATTN_OK", 1: "ATTN_ERR_NULL", 2: "ATTN_ERR_SHAPE", 3: "ATTN_ERR_ALIGN",
+                4: "ATTN_ERR_UNSUPPORTED", 5: "ATTN_ERR_CUDA", 6: "ATTN_ERR_DEVICE_TIMEOUT",
+                7: "ATTN_ERR_WORKSPACE"}
+
+_lib = None
+
+
+class AttnError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__("%s: %s" % (what, status_string(status) if _lib else STATUS_NAMES.get(status)))
+
+
+def load() -> ctypes.CDLL:
+    """Load libattn_b200.so from the package folder (raises if it is not built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError("libattn_b200.so is not built (run `python -m "
+                           "dnn_compiler_pipelining_b200.build`); there is no fallback path")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i, u64, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_uint64, ctypes.c_size_t
+    lib.attn_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, vp]
+    lib.attn_fwd.restype = i
+    lib.attn_fwd_host.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, vp, sz, vp]
+    lib.attn_fwd_host.restype = i
+    lib.attn_fwd_host_workspace_bytes.argtypes = [i, i, i, i, i]
+    lib.attn_fwd_host_workspace_bytes.restype = sz
+    lib.attn_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32)]
+    lib.attn_device_status.restype = i
+    lib.attn_set_wait_timeout_ns.argtypes = [u64]
+    lib.attn_set_wait_timeout_ns.restype = u64
+    lib.attn_selftest_wait_timeout.argtypes = [u64, vp]
+    lib.attn_selftest_wait_timeout.restype = i
+    lib.attn_status_string.argtypes = [i]
+    lib.attn_status_string.restype = ctypes.c_char_p
+    lib.attn_version.argtypes = []
+    lib.attn_version.restype = i
+    _lib = lib
+    return lib
+
+
+def status_string(status: int) -> str:
+    return load().attn_status_string(int(status)).decode()
+
+
+def version() -> int:
+    return int(load().attn_version())
+
+
+def _stream_ptr(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream)
+
+
+def _check_dev(t: torch.Tensor, name: str, dtype):
+    if not (t.is_cuda and t.dtype == dtype and t.is_contiguous()):
+        raise ValueError("%s must be a contiguous CUDA %s tensor" % (name, dtype))
+
+
+def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = True,
+             o: torch.Tensor | None = None, lse: torch.Tensor | None = None, stream=None):
+    """O, LSE = attention(Q, K, V) on the GPU through the C ABI.
+
+    q: [B,Hq,S,D] fp16; k, v: [B,Hkv,S,D] fp16 (contiguous, on the current
+    device).  Returns (o [B,Hq,S,D] fp16, lse [B,Hq,S] fp32); o / lse may be
+    passed in preallocated.  Asynchronous on ``stream`` (default: the current
+    torch stream).
+    """
+    lib = load()
+    _check_dev(q, "q", torch.float16)
+    _check_dev(k, "k", torch.float16)
+    _check_dev(v, "v", torch.float16)
+    B, Hq, S, D = q.shape
+    Hkv = k.shape[1]
+    if tuple(k.shape) != (B, Hkv, S, D) or tuple(v.shape) != tuple(k.shape):
+        raise ValueError("shape mismatch: q %s k %s v %s" % (tuple(q.shape), tuple(k.shape),
+                                                             tuple(v.shape)))
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, S), dtype=torch.float32, device=q.device)
+    _check_dev(o, "o", torch.float16)
+    _check_dev(lse, "lse", torch.float32)
+    st = lib.attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                      B, Hq, Hkv, S, D, int(bool(causal)), _stream_ptr(stream))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_fwd")
+    return o, lse
+
+
+def attn_fwd_raw(q_ptr: int, k_ptr: int, v_ptr: int, o_ptr: int, lse_ptr: int, B: int, Hq: int,
+                 Hkv: int, S: int, D: int, causal: bool, stream_ptr: int) -> int:
+    """The C entry point with raw addresses; returns the status code."""
+    return int(load().attn_fwd(q_ptr, k_ptr, v_ptr, o_ptr, lse_ptr, B, Hq, Hkv, S, D,
+                               int(bool(causal)), stream_ptr))
+
+
+def host_workspace_bytes(B: int, Hq: int, Hkv: int, S: int, D: int) -> int:
+    return int(load().attn_fwd_host_workspace_bytes(B, Hq, Hkv, S, D))
+
+
+def attn_fwd_host(q_h: torch.Tensor, k_h: torch.Tensor, v_h: torch.Tensor, o_h: torch.Tensor,
+                  lse_h: torch.Tensor, causal: bool, workspace: torch.Tensor, stream=None):
+    """Host-buffer entry: CPU tensors in and out, device workspace from the caller.
+    Synchronizes the stream before returning."""
+    lib = load()
+    for t, n in ((q_h, "q"), (k_h, "k"), (v_h, "v"), (o_h, "o"), (lse_h, "lse")):
+        if t.is_cuda or not t.is_contiguous():
+            raise ValueError("%s must be a contiguous CPU tensor" % n)
+    B, Hq, S, D = q_h.shape
+    Hkv = k_h.shape[1]
+    st = lib.attn_fwd_host(q_h.data_ptr(), k_h.data_ptr(), v_h.data_ptr(), o_h.data_ptr(),
+                           lse_h.data_ptr(), B, Hq, Hkv, S, D, int(bool(causal)),
+                           workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                           _stream_ptr(stream))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_fwd_host")
+
+
+def device_status(stream=None):
+    """(status, site): synchronizes, reads and clears the device status word."""
+    site = ctypes.c_uint32(0)
+    st = load().attn_device_status(_stream_ptr(stream), ctypes.byref(site))
+    return int(st), int(site.value)
+
+
+def set_wait_timeout_ns(ns: int) -> int:
+    return int(load().attn_set_wait_timeout_ns(int(ns)))
+
+
+def selftest_wait_timeout(ns: int, stream=None) -> int:
+    return int(load().attn_selftest_wait_timeout(int(ns), _stream_ptr(stream)))

@@ -1,0 +1,250 @@
+// attn_api.cu -- C ABI of libattn_b200.so (declared in include/attn.h):
+// argument validation, TMA tensor-map encoding, kernel launch, the
+// per-device status word, the host-buffer entry point and the bounded-wait
+// self-test.  Nothing here allocates device memory.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "attn.h"
+#include "attn_fwd_sm100.cuh"
+
+namespace attn_b200 {
+namespace {
+
+constexpr int kStagesV1 = 2;
+constexpr int kMaxDevices = 64;
+
+std::atomic<uint64_t> g_timeout_ns{2000000000ull};
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult qres;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault,
+                                         &qres) == cudaSuccess &&
+        qres == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+// Per-device one-time setup: architecture check and the kernel's shared
+// memory opt-in.  0 = not done, 1 = ok, 2 = unsupported device.
+std::atomic<int> g_dev_state[kMaxDevices];
+std::mutex g_dev_mutex;
+
+template <int kStages>
+size_t v1_smem_bytes() {
+  return sizeof(SharedV1<kStages>) + 1024;  // + slack to align the base to 1 KiB
+}
+
+attn_status device_setup(int* dev_out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return ATTN_ERR_UNSUPPORTED;
+  *dev_out = dev;
+  int st = g_dev_state[dev].load(std::memory_order_acquire);
+  if (st == 1) return ATTN_OK;
+  if (st == 2) return ATTN_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_dev_mutex);
+  st = g_dev_state[dev].load(std::memory_order_acquire);
+  if (st == 0) {
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+      return ATTN_ERR_CUDA;
+    if (major != 10 || minor != 0) {
+      g_dev_state[dev].store(2, std::memory_order_release);
+      return ATTN_ERR_UNSUPPORTED;
+    }
+    if (cudaFuncSetAttribute(attn_fwd_v1_kernel<kStagesV1>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(v1_smem_bytes<kStagesV1>())) != cudaSuccess)
+      return ATTN_ERR_CUDA;
+    g_dev_state[dev].store(1, std::memory_order_release);
+  }
+  return g_dev_state[dev].load() == 1 ? ATTN_OK : ATTN_ERR_UNSUPPORTED;
+}
+
+// 2-D view [rows, 128] fp16 of a dense [.., S, 128] tensor; 64 x 128 boxes
+// (one 128-byte swizzle panel of 128 rows).
+bool encode_rows_map(CUtensorMap* map, const void* base, uint64_t rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(kHeadDim), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(kHeadDim) * 2};
+  cuuint32_t box[2] = {64, static_cast<cuuint32_t>(kBlockM)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+attn_status validate_sizes(int B, int Hq, int Hkv, int S, int D) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || S < 1 || D < 1) return ATTN_ERR_SHAPE;
+  if (Hq % Hkv != 0) return ATTN_ERR_SHAPE;
+  if (D != kHeadDim) return ATTN_ERR_UNSUPPORTED;
+  if (S % kBlockM != 0) return ATTN_ERR_UNSUPPORTED;
+  // row indices are 32-bit signed in the kernel and in TMA coordinates
+  const int64_t q_rows = static_cast<int64_t>(B) * Hq * S;
+  if (q_rows >= (int64_t(1) << 31)) return ATTN_ERR_SHAPE;
+  if (Hq > 65535 || B > 65535) return ATTN_ERR_SHAPE;  // grid y / z limits
+  return ATTN_OK;
+}
+
+size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+}  // namespace
+}  // namespace attn_b200
+
+using namespace attn_b200;
+
+extern "C" {
+
+int attn_version(void) { return (1 << 16) | 0; }
+
+const char* attn_status_string(attn_status s) {
+  switch (s) {
+    case ATTN_OK: return "ATTN_OK";
+    case ATTN_ERR_NULL: return "ATTN_ERR_NULL: a required pointer is NULL";
+    case ATTN_ERR_SHAPE: return "ATTN_ERR_SHAPE: invalid or too large sizes";
+    case ATTN_ERR_ALIGN: return "ATTN_ERR_ALIGN: a device pointer is not 16-byte aligned";
+    case ATTN_ERR_UNSUPPORTED:
+      return "ATTN_ERR_UNSUPPORTED: needs D == 128, S % 128 == 0 and an sm_100 device";
+    case ATTN_ERR_CUDA: return "ATTN_ERR_CUDA: a CUDA call failed";
+    case ATTN_ERR_DEVICE_TIMEOUT: return "ATTN_ERR_DEVICE_TIMEOUT: a kernel wait ran out";
+    case ATTN_ERR_WORKSPACE: return "ATTN_ERR_WORKSPACE: device workspace too small";
+  }
+  return "ATTN_ERR_UNKNOWN";
+}
+
+uint64_t attn_set_wait_timeout_ns(uint64_t ns) {
+  if (ns < 1000000ull) ns = 1000000ull;
+  return g_timeout_ns.exchange(ns);
+}
+
+attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                     int Hq, int Hkv, int S, int D, int causal, void* stream) {
+  if (!q || !k || !v || !o || !lse) return ATTN_ERR_NULL;
+  attn_status st = validate_sizes(B, Hq, Hkv, S, D);
+  if (st != ATTN_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+    return ATTN_ERR_ALIGN;
+  int dev = 0;
+  st = device_setup(&dev);
+  if (st != ATTN_OK) return st;
+
+  CUtensorMap tm_q, tm_k, tm_v;
+  if (!encode_rows_map(&tm_q, q, static_cast<uint64_t>(B) * Hq * S) ||
+      !encode_rows_map(&tm_k, k, static_cast<uint64_t>(B) * Hkv * S) ||
+      !encode_rows_map(&tm_v, v, static_cast<uint64_t>(B) * Hkv * S))
+    return ATTN_ERR_CUDA;
+
+  FwdParams p;
+  p.o = static_cast<__half*>(o);
+  p.lse = lse;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.S = S;
+  p.causal = causal ? 1 : 0;
+  p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
+  p.timeout_ns = g_timeout_ns.load();
+
+  dim3 grid(S / kBlockM, Hq, B);
+  dim3 block(192);
+  attn_fwd_v1_kernel<kStagesV1><<<grid, block, v1_smem_bytes<kStagesV1>(),
+                                  static_cast<cudaStream_t>(stream)>>>(tm_q, tm_k, tm_v, p);
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  return ATTN_OK;
+}
+
+size_t attn_fwd_host_workspace_bytes(int B, int Hq, int Hkv, int S, int D) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || S < 1 || D < 1) return 0;
+  const size_t q = static_cast<size_t>(B) * Hq * S * D * 2;
+  const size_t kv = static_cast<size_t>(B) * Hkv * S * D * 2;
+  const size_t l = static_cast<size_t>(B) * Hq * S * 4;
+  return round256(q) * 2 + round256(kv) * 2 + round256(l);
+}
+
+attn_status attn_device_status(void* stream, uint32_t* site) {
+  if (site) *site = 0;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return ATTN_ERR_CUDA;
+  unsigned int words[2] = {0, 0};
+  if (cudaMemcpyFromSymbol(words, g_attn_status, sizeof(words)) != cudaSuccess) return ATTN_ERR_CUDA;
+  if (words[0] != 0 || words[1] != 0) {
+    const unsigned int zero[2] = {0, 0};
+    if (cudaMemcpyToSymbol(g_attn_status, zero, sizeof(zero)) != cudaSuccess) return ATTN_ERR_CUDA;
+  }
+  if (site) *site = words[1];
+  return (words[0] & kStatusTimeout) ? ATTN_ERR_DEVICE_TIMEOUT : ATTN_OK;
+}
+
+attn_status attn_fwd_host(const void* q_h, const void* k_h, const void* v_h, void* o_h,
+                          float* lse_h, int B, int Hq, int Hkv, int S, int D, int causal,
+                          void* workspace, size_t workspace_bytes, void* stream) {
+  if (!q_h || !k_h || !v_h || !o_h || !lse_h || !workspace) return ATTN_ERR_NULL;
+  attn_status st = validate_sizes(B, Hq, Hkv, S, D);
+  if (st != ATTN_OK) return st;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return ATTN_ERR_ALIGN;
+  const size_t need = attn_fwd_host_workspace_bytes(B, Hq, Hkv, S, D);
+  if (workspace_bytes < need) return ATTN_ERR_WORKSPACE;
+  const size_t qb = static_cast<size_t>(B) * Hq * S * D * 2;
+  const size_t kvb = static_cast<size_t>(B) * Hkv * S * D * 2;
+  const size_t lb = static_cast<size_t>(B) * Hq * S * 4;
+  char* w = static_cast<char*>(workspace);
+  char* dq = w;
+  char* dk = dq + round256(qb);
+  char* dv = dk + round256(kvb);
+  char* dout = dv + round256(kvb);
+  float* dl = reinterpret_cast<float*>(dout + round256(qb));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(dq, q_h, qb, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaMemcpyAsync(dk, k_h, kvb, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaMemcpyAsync(dv, v_h, kvb, cudaMemcpyHostToDevice, s) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  st = attn_fwd(dq, dk, dv, dout, dl, B, Hq, Hkv, S, D, causal, stream);
+  if (st != ATTN_OK) return st;
+  if (cudaMemcpyAsync(o_h, dout, qb, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaMemcpyAsync(lse_h, dl, lb, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  return attn_device_status(stream, nullptr);
+}
+
+}  // extern "C"
+
+namespace attn_b200 {
+// One thread waits, with the kernels' bounded wait, on an mbarrier that no
+// one arrives on.
+__global__ void selftest_wait_kernel(uint64_t timeout_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_addr(&bar), 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(smem_addr(&bar), 0, &abort_flag, timeout_ns, 0x501);
+}
+}  // namespace attn_b200
+
+extern "C" attn_status attn_selftest_wait_timeout(uint64_t timeout_ns, void* stream) {
+  int dev = 0;
+  attn_status st = device_setup(&dev);
+  if (st != ATTN_OK) return st;
+  selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(timeout_ns);
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  return attn_device_status(stream, nullptr);
+}

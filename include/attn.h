@@ -1,0 +1,132 @@
+/*
+ * attn.h -- C ABI of the B200 (sm_100a) fused attention forward library
+ *           libattn_b200.so.
+ *
+ * Operation (attn_fwd).  Scaled dot-product attention with grouped-query
+ * heads and an optional causal mask, computed in one fused pass that never
+ * writes the S x S score matrix to memory.  This is the FlashAttention forward
+ * that the PipeThreader pages evaluate on LLaMA3-8B/70B head shapes, SEQ
+ * 512-8k and batch 1/64 (papers.lqhl.me "PipeThreader-OSDI25", section
+ * 实验与结果, paper Sec. 6.2 / Fig. 12), and whose TMA-load / tensor-core /
+ * CUDA-core task split those pages describe (section 核心方法, "sTask / sEU").
+ * The pages do not print the formula; the textbook definition is used:
+ *
+ *   g          = hq / (Hq / Hkv)            (contiguous groups of query heads)
+ *   s_ij       = <Q[b,hq,i,:], K[b,g,j,:]> / sqrt(D),  j in A(i)
+ *   A(i)       = {0..i} if causal else {0..S-1}
+ *   O[b,hq,i,:] = sum_j softmax_j(s_i.) V[b,g,j,:]
+ *   LSE[b,hq,i] = ln sum_{j in A(i)} exp(s_ij)   (natural log, scaled logits)
+ *
+ * Precision: Q, K, V and O are IEEE fp16; products accumulate in fp32; the
+ * probabilities feed the second product as fp16; LSE is fp32.
+ *
+ * Conventions shared by every entry point:
+ *   - Layouts are dense row-major: Q, O [B, Hq, S, D]; K, V [B, Hkv, S, D];
+ *     LSE [B, Hq, S].  "Device" pointers are CUDA device (or managed)
+ *     addresses on the current device; "host" pointers are CPU addresses.
+ *   - The caller owns every buffer.  The library never allocates device or
+ *     host memory in these calls and keeps no pointer after returning.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls
+ *     are asynchronous with respect to the host unless stated otherwise.
+ *   - Arguments are validated before anything is launched; a rejected call
+ *     launches nothing and leaves the outputs untouched.
+ *   - Every wait inside the kernels is bounded in time.  A wait that runs out
+ *     makes the kernel stop early (without faulting) and records
+ *     ATTN_ERR_DEVICE_TIMEOUT in a per-device status word, read back with
+ *     attn_device_status().
+ */
+#ifndef ATTN_B200_H
+#define ATTN_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum attn_status {
+  ATTN_OK = 0,
+  ATTN_ERR_NULL = 1,           /* a required pointer is NULL */
+  ATTN_ERR_SHAPE = 2,          /* B,Hq,Hkv,S < 1, Hq % Hkv != 0, or a size overflows */
+  ATTN_ERR_ALIGN = 3,          /* a device pointer is not 16-byte aligned */
+  ATTN_ERR_UNSUPPORTED = 4,    /* D != 128, S % 128 != 0, or not an sm_100 device */
+  ATTN_ERR_CUDA = 5,           /* a CUDA runtime / driver call failed */
+  ATTN_ERR_DEVICE_TIMEOUT = 6, /* a kernel wait ran out; results are invalid */
+  ATTN_ERR_WORKSPACE = 7       /* the device workspace given is too small */
+} attn_status;
+
+/*
+ * attn_fwd -- fused attention forward on device buffers.
+ *   q   : device, fp16 [B, Hq, S, D], 16-byte aligned, read only.
+ *   k, v: device, fp16 [B, Hkv, S, D], 16-byte aligned, read only.
+ *   o   : device, fp16 [B, Hq, S, D], 16-byte aligned, written.
+ *   lse : device, fp32 [B, Hq, S], 16-byte aligned, written (must not be NULL).
+ *   B, Hq, Hkv, S, D: sizes; Hq % Hkv == 0; D == 128; S % 128 == 0.
+ *   causal: nonzero for the causal mask j <= i (square, Sq == Sk == S).
+ *   stream: cudaStream_t to launch on.
+ * Returns ATTN_OK once the kernel is enqueued; errors as listed above.  The
+ * outputs must not overlap the inputs.
+ */
+attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                     int B, int Hq, int Hkv, int S, int D, int causal, void* stream);
+
+/*
+ * attn_fwd_host_workspace_bytes -- size in bytes of the device workspace that
+ * attn_fwd_host needs for these sizes (Q, K, V, O and LSE, each rounded up to
+ * 256 bytes).  Returns 0 for invalid sizes.
+ */
+size_t attn_fwd_host_workspace_bytes(int B, int Hq, int Hkv, int S, int D);
+
+/*
+ * attn_fwd_host -- the same operation on HOST buffers, for callers whose data
+ * live in CPU memory.  q_h, k_h, v_h (fp16, layouts as above) are copied into
+ * the caller's device workspace, attn_fwd runs there, and O and LSE are
+ * copied back into o_h (fp16) and lse_h (fp32).  All copies and the kernel
+ * are enqueued on `stream`, and the call synchronizes the stream before it
+ * returns, so the host buffers hold the results on ATTN_OK.  Host buffers may
+ * be pageable or pinned (pinned copies run asynchronously and faster).
+ *   workspace: device, >= attn_fwd_host_workspace_bytes(...) bytes, 256-byte
+ *              aligned; its contents are overwritten.
+ * Also returns ATTN_ERR_DEVICE_TIMEOUT if the kernel reported one.
+ */
+attn_status attn_fwd_host(const void* q_h, const void* k_h, const void* v_h, void* o_h,
+                          float* lse_h, int B, int Hq, int Hkv, int S, int D, int causal,
+                          void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * attn_device_status -- synchronizes `stream`, then reads and clears the
+ * current device's status word.  Returns ATTN_ERR_DEVICE_TIMEOUT if any
+ * kernel of this library recorded a timed-out wait since the last read,
+ * ATTN_ERR_CUDA if synchronizing failed, else ATTN_OK.  `site`, if not NULL,
+ * receives the first recorded wait site (0 when none).
+ */
+attn_status attn_device_status(void* stream, uint32_t* site);
+
+/*
+ * attn_set_wait_timeout_ns -- bound, in nanoseconds, on every wait inside the
+ * kernels launched afterwards from this process (default 2e9 = 2 s; values
+ * below 1e6 are raised to 1e6).  Returns the previous value.
+ */
+uint64_t attn_set_wait_timeout_ns(uint64_t ns);
+
+/*
+ * attn_selftest_wait_timeout -- launches one CTA that waits on an mbarrier
+ * nothing will ever complete, with a bound of timeout_ns, using the same
+ * bounded-wait routine as the attention kernels.  Synchronizes `stream` and
+ * returns what attn_device_status() then reports (ATTN_ERR_DEVICE_TIMEOUT when
+ * the bound works).  The GPU context stays usable afterwards.
+ */
+attn_status attn_selftest_wait_timeout(uint64_t timeout_ns, void* stream);
+
+/* Human-readable name of a status code (static storage, never NULL). */
+const char* attn_status_string(attn_status status);
+
+/* Library ABI version: (major << 16) | minor. */
+int attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATTN_B200_H */
