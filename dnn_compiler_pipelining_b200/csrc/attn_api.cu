@@ -9,7 +9,9 @@
 #include <atomic>
 #include <cmath>
 #include <cstdint>
+#include <map>
 #include <mutex>
+#include <utility>
 
 #include "attn.h"
 #include "attn_fwd_sm100.cuh"
@@ -17,7 +19,6 @@
 namespace attn_b200 {
 namespace {
 
-constexpr int kStagesV1 = 2;
 constexpr int kMaxDevices = 64;
 
 std::atomic<uint64_t> g_timeout_ns{2000000000ull};
@@ -39,11 +40,37 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 // Per-device one-time setup: architecture check and the kernel's shared
 // memory opt-in.  0 = not done, 1 = ok, 2 = unsupported device.
 std::atomic<int> g_dev_state[kMaxDevices];
+int g_dev_sms[kMaxDevices];
 std::mutex g_dev_mutex;
 
-template <int kStages>
-size_t v1_smem_bytes() {
-  return sizeof(SharedV1<kStages>) + 1024;  // + slack to align the base to 1 KiB
+// Redo lists (items the fast pass hands to the hi+lo pass), one per
+// (device, stream): launches on one stream run in order, so a list is never
+// shared by launches that could overlap.
+constexpr unsigned int kRedoCapacity = 1u << 16;
+std::map<std::pair<int, cudaStream_t>, unsigned int*> g_redo_lists;
+std::mutex g_redo_mutex;
+
+size_t redo_bytes() { return (kRedoHeaderWords + kRedoCapacity) * sizeof(unsigned int); }
+
+// Returns the list for (dev, stream), allocating and zeroing it (on that
+// stream) the first time.
+unsigned int* redo_list(int dev, cudaStream_t stream) {
+  std::lock_guard<std::mutex> lock(g_redo_mutex);
+  auto key = std::make_pair(dev, stream);
+  auto it = g_redo_lists.find(key);
+  if (it != g_redo_lists.end()) return it->second;
+  void* ptr = nullptr;
+  if (cudaMalloc(&ptr, redo_bytes()) != cudaSuccess) return nullptr;
+  if (cudaMemsetAsync(ptr, 0, redo_bytes(), stream) != cudaSuccess) {
+    cudaFree(ptr);
+    return nullptr;
+  }
+  g_redo_lists[key] = static_cast<unsigned int*>(ptr);
+  return static_cast<unsigned int*>(ptr);
+}
+
+size_t fwd_smem_bytes() {
+  return sizeof(SharedFwd) + 1024;  // + slack to align the base to 1 KiB
 }
 
 attn_status device_setup(int* dev_out) {
@@ -65,9 +92,11 @@ attn_status device_setup(int* dev_out) {
       g_dev_state[dev].store(2, std::memory_order_release);
       return ATTN_ERR_UNSUPPORTED;
     }
-    if (cudaFuncSetAttribute(attn_fwd_v1_kernel<kStagesV1>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(v1_smem_bytes<kStagesV1>())) != cudaSuccess)
+    if (cudaDeviceGetAttribute(&g_dev_sms[dev], cudaDevAttrMultiProcessorCount, dev) !=
+        cudaSuccess)
+      return ATTN_ERR_CUDA;
+    if (cudaFuncSetAttribute(attn_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(fwd_smem_bytes())) != cudaSuccess)
       return ATTN_ERR_CUDA;
     g_dev_state[dev].store(1, std::memory_order_release);
   }
@@ -159,13 +188,25 @@ attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float
   p.Hkv = Hkv;
   p.S = S;
   p.causal = causal ? 1 : 0;
+  p.n_qb = S / kBlockM;
+  p.n_qb2 = (p.n_qb + 1) / 2;
+  p.group = Hq / Hkv;
+  p.n_items = B * Hq * p.n_qb2;
   p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
   p.timeout_ns = g_timeout_ns.load();
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  p.redo = redo_list(dev, cs);
+  if (!p.redo) return ATTN_ERR_CUDA;
+  p.redo_capacity = kRedoCapacity;
 
-  dim3 grid(S / kBlockM, Hq, B);
-  dim3 block(192);
-  attn_fwd_v1_kernel<kStagesV1><<<grid, block, v1_smem_bytes<kStagesV1>(),
-                                  static_cast<cudaStream_t>(stream)>>>(tm_q, tm_k, tm_v, p);
+  // fast pass over every item, then the hi+lo pass over the items it listed
+  const int sms = g_dev_sms[dev];
+  p.mode = 0;
+  attn_fwd_kernel<<<p.n_items < sms ? p.n_items : sms, kThreads, fwd_smem_bytes(), cs>>>(tm_q, tm_k,
+                                                                                       tm_v, p);
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  p.mode = 1;
+  attn_fwd_kernel<<<sms, kThreads, fwd_smem_bytes(), cs>>>(tm_q, tm_k, tm_v, p);
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
   return ATTN_OK;
 }

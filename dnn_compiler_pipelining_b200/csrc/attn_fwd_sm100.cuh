@@ -1,34 +1,46 @@
 // attn_fwd_sm100.cuh -- fused attention forward for sm_100a (B200).
 //
 // One pass computes O = softmax(Q K^T / sqrt(D) [+ causal mask]) V and the
-// row log-sum-exp, for grouped-query heads, without writing the score matrix
-// to memory.  This is the FlashAttention forward that the PipeThreader pages
-// evaluate (papers.lqhl.me "PipeThreader-OSDI25", section 实验与结果, paper
-// Sec. 6.2 / Fig. 12).  Their pipeline (section 核心方法, "sTask / sEU") splits
-// the operator into load, mma and softmax tasks on TMA, TensorCore and CUDA
-// cores and overlaps them inside an SM; here that split is fixed by hand as
-// warp roles:
+// row log-sum-exp for grouped-query heads, without writing the score matrix
+// to memory: the FlashAttention forward that the PipeThreader pages evaluate
+// (papers.lqhl.me "PipeThreader-OSDI25", section 实验与结果, paper Sec. 6.2 /
+// Fig. 12).  The pages build it from load, mma and softmax tasks on TMA,
+// TensorCore and CUDA-core units overlapped inside an SM (section 核心方法,
+// "sTask / sEU"; dependences kept by barrier-sTasks, "sTask-graph ->
+// sProgram").  Here that split is fixed by hand for B200:
 //
-//   warp 4       TMA producer: Q tile once, then K_j / V_j tiles into a ring
-//                of kStages shared-memory stages.
-//   warp 5       MMA issuer (one thread): S_j = Q K_j^T into TMEM, then
-//                O += P_j V_j with P read from TMEM; tcgen05.commit signals
-//                mbarriers when they finish.
-//   warps 0..3   softmax, one query row per thread (TMEM lane = row): load
-//                S_j, apply the causal mask on the diagonal tile, update the
-//                running max, exponentiate, write P_j (fp16) over S_j in
-//                TMEM; rescale O when the running max grew by more than
-//                kRescaleLog2 (lazy rescaling is exact: O and the row sum l
-//                always share the same reference max); finally O / l and
-//                LSE.
+// Persistent kernel, one CTA per SM.  A work item is 256 query rows of one
+// (batch, query head): two 128-row tiles, A and B, that share every K/V tile
+// and take turns on the tensor core, so one tile's softmax runs while the
+// other tile's MMAs do.  Items are ordered kv-head by kv-head (the query
+// heads of a group and all their row blocks close together, so K/V stay in
+// L2) and handed out round-robin to the CTAs.
 //
-// TMEM (512 columns): S/P buffer 0 at [0,128), buffer 1 at [128,256),
-// O at [256,384).  Two S buffers let the tensor core compute S_{j+1} while
-// the softmax works on S_j.
+// Warp roles (512 threads, registers re-split with setmaxnreg):
+//   warps 0-3   softmax of tile A   (one query row per thread = TMEM lane)
+//   warps 4-7   softmax of tile B
+//   warps 8-11  epilogue: O / l -> fp16, LSE, for both tiles
+//   warp 12     TMA producer: Q_A, Q_B per item, K_j / V_j into a ring
+//   warp 13     MMA issuer (one thread): S_X = Q_X K_j^T, O_X += P_X V_j
+//   warps 14-15 idle
 //
-// Shared memory tiles are 128 rows x 128 fp16 stored as two 64-column panels
-// of 16 KiB in the TMA 128-byte swizzle, which is also the tcgen05 "SW128"
-// canonical layout: Q and K are K-major operands, V is an MN-major operand.
+// TMEM (512 columns): S_A [0,128), S_B [128,256), O_A [256,384),
+// O_B [384,512).  P_X (fp16) is written over the first 64 columns of S_X
+// (and, in the redo pass, its low half over the next 64).
+//
+// Per tile X and key block j the MMA thread issues PV_X(j-1) and then
+// S_X(j); tcgen05 operations complete in order, so when S_X(j) signals
+// s_full, O_X already holds P_X(j-1) V_{j-1} and the softmax may rescale it.
+//
+// Numerics: P is rounded to fp16 and the row sum l accumulates exactly those
+// rounded values, so O / l uses one consistent set of weights.  Lazy
+// rescaling keeps a reference max per row and rescales O only when the row
+// max grows by more than 2^kRescaleLog2 (exact: O and l share the
+// reference).  The output is rounded to fp16, whose half-ulp for |O| >= 4 is
+// 1.95e-3, so rows there need more than fp16 weights can give.  The fast
+// pass (mode 0) therefore records each item with a row max|O| >=
+// kRedoThreshold, and a second launch (mode 1) recomputes just those items
+// with P split as hi + lo fp16 (about 22-bit weights, one extra PV MMA).
 #pragma once
 
 #include <cuda_fp16.h>
@@ -38,321 +50,565 @@
 namespace attn_b200 {
 
 constexpr int kBlockM = 128;   // query rows per tile
-constexpr int kBlockN = 128;   // keys per tile
+constexpr int kBlockN = 128;   // keys per K/V tile
 constexpr int kHeadDim = 128;  // D
+constexpr int kItemRows = 2 * kBlockM;
+constexpr int kStages = 2;     // K/V ring depth
+constexpr int kThreads = 512;
 constexpr uint32_t kTileBytes = kBlockM * kHeadDim * 2;  // 32 KiB fp16 tile
-constexpr uint32_t kPanelBytes = kTileBytes / 2;         // 64-column swizzle panel
-constexpr float kRescaleLog2 = 8.0f;  // rescale O only when the max grows by > 2^8
+constexpr uint32_t kPanelBytes = kTileBytes / 2;         // one 64-column swizzle panel
+constexpr float kRescaleLog2 = 8.0f;
+constexpr float kRedoThreshold = 3.98f;
 constexpr float kLn2 = 0.69314718055994531f;
+
+constexpr int kEpilogueWarp0 = 8;
+constexpr int kProducerWarp = 12;
+constexpr int kMmaWarp = 13;
+constexpr int kRegsSoftmax = 192;
+constexpr int kRegsEpilogue = 64;
+constexpr int kRegsOther = 64;
+static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsEpilogue + 128 * kRegsOther <= kThreads * 128,
+              "register split exceeds the launch allocation");
+
+constexpr uint32_t kTmemCols = 512;
+__device__ __forceinline__ uint32_t tmem_s_col(int x) { return x * 128u; }
+__device__ __forceinline__ uint32_t tmem_o_col(int x) { return 256u + x * 128u; }
+
+// redo list (device scratch): header {count, done, -, -} then item ids
+constexpr int kRedoHeaderWords = 4;
 
 struct FwdParams {
   __half* o;
   float* lse;
   int B, Hq, Hkv, S;
   int causal;
+  int mode;          // 0: fast pass; 1: redo listed items with hi+lo P
+  int n_items;       // B * Hq * n_qb2
+  int n_qb;          // S / 128 row blocks
+  int n_qb2;         // ceil(n_qb / 2) items per (batch, head)
+  int group;         // Hq / Hkv
   float scale_log2;  // log2(e) / sqrt(D)
   unsigned long long timeout_ns;
+  unsigned int* redo;  // redo list
+  unsigned int redo_capacity;
 };
 
-// wait sites recorded in the status word when a bounded wait runs out
 enum WaitSite : uint32_t {
-  kSiteProducerEmpty = 0x101,
+  kSiteProducerQ = 0x101,
+  kSiteProducerKV = 0x102,
   kSiteMmaQ = 0x201,
   kSiteMmaK = 0x202,
-  kSiteMmaP = 0x203,
-  kSiteMmaV = 0x204,
+  kSiteMmaV = 0x203,
+  kSiteMmaP = 0x204,
+  kSiteMmaO = 0x205,
   kSiteSoftmaxS = 0x301,
-  kSiteSoftmaxO = 0x302,
-  kSiteEpilogueO = 0x303,
+  kSiteEpilogueO = 0x401,
+  kSiteEpilogueStats = 0x402,
+  kSiteDrain = 0x501,
 };
 
-template <int kStages>
-struct alignas(1024) SharedV1 {
-  uint8_t q[kTileBytes];
+struct alignas(1024) SharedFwd {
+  uint8_t q[2][kTileBytes];
   uint8_t k[kStages][kTileBytes];
   uint8_t v[kStages][kTileBytes];
-  uint64_t q_full;
-  uint64_t k_full[kStages];
-  uint64_t v_full[kStages];
-  uint64_t kv_empty[kStages];
-  uint64_t s_full[2];
-  uint64_t p_full[2];
-  uint64_t pv_done[2];
+  float stat_m[2][2][kBlockM];  // [parity of the tile's active-item count][tile][row]
+  float stat_l[2][2][kBlockM];
+  uint64_t q_full, q_empty;
+  uint64_t k_full[kStages], v_full[kStages], kv_empty[kStages];
+  uint64_t s_full[2], p_full[2], o_done[2], o_free[2], stats_ready[2];
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
+  int item_flag[2];   // [item parity]: a row of the item needs the redo pass
+  int item_warps[2];  // [item parity]: epilogue warps done with the item
+  unsigned int n_listed;
 };
 
-constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kTmemO = 256;
+struct Item {
+  int b, hq, g, qb2;
+  int n_kv[2];   // key blocks of tile A, tile B (0: tile B lies past the end)
+  int n_blocks;  // max of the two
+};
 
-// Waits that must finish even after another role gave up (in-flight copies
-// and MMAs complete on their own); bounded all the same.
-__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64_t timeout_ns) {
-  int never = 0;
-  mbar_wait(bar, parity, &never, timeout_ns, 0x401);
+__device__ __forceinline__ Item decode_item(const FwdParams& p, int id) {
+  // kv-head major; inside a kv head: row blocks from last to first, the
+  // group's query heads adjacent
+  const int per_kv = p.group * p.n_qb2;
+  const int kvh = id / per_kv;
+  const int rem = id - kvh * per_kv;
+  Item it;
+  it.b = kvh / p.Hkv;
+  it.g = kvh - it.b * p.Hkv;
+  it.qb2 = p.n_qb2 - 1 - rem / p.group;
+  it.hq = it.g * p.group + rem % p.group;
+  const bool b_active = 2 * it.qb2 + 1 < p.n_qb;
+  if (p.causal) {
+    it.n_kv[0] = 2 * it.qb2 + 1;
+    it.n_kv[1] = b_active ? 2 * it.qb2 + 2 : 0;
+  } else {
+    it.n_kv[0] = p.n_qb;
+    it.n_kv[1] = b_active ? p.n_qb : 0;
+  }
+  it.n_blocks = it.n_kv[1] > it.n_kv[0] ? it.n_kv[1] : it.n_kv[0];
+  return it;
 }
 
-template <int kStages>
-__global__ void __launch_bounds__(192, 1)
-    attn_fwd_v1_kernel(const __grid_constant__ CUtensorMap tm_q,
-                       const __grid_constant__ CUtensorMap tm_k,
-                       const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
-  using Smem = SharedV1<kStages>;
+// k-th work item of this CTA, or -1 when done.
+__device__ __forceinline__ int work_item(const FwdParams& p, int k, unsigned int n_listed) {
+  const long long idx = static_cast<long long>(blockIdx.x) + static_cast<long long>(k) * gridDim.x;
+  if (p.mode == 1 && n_listed <= p.redo_capacity) {
+    if (idx >= n_listed) return -1;
+    const unsigned int id = p.redo[kRedoHeaderWords + idx];
+    // an id from another call's list (left by a launch that failed) is
+    // replaced by item 0: recomputing a valid item is always harmless
+    return id < static_cast<unsigned int>(p.n_items) ? static_cast<int>(id) : 0;
+  }
+  return idx < p.n_items ? static_cast<int>(idx) : -1;
+}
+
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64_t timeout_ns) {
+  int never = 0;
+  mbar_wait(bar, parity, &never, timeout_ns, kSiteDrain);
+}
+
+__device__ __forceinline__ uint32_t ring_parity(int rc) { return (rc / kStages) & 1; }
+
+// S_X(j) = Q_X K^T: 8 MMAs of K = 16 over the head dimension.  Both operands
+// are K-major; 16 columns are 32 bytes inside a 128-byte swizzled row and
+// columns 64..127 live in the second panel.
+// A descriptor's start address sits in its low bits (16-byte units), so a
+// descriptor for base + off is the base descriptor plus off >> 4 (shared
+// memory offsets stay below 256 KiB, so no carry leaves the field).
+template <int kk>
+__device__ __forceinline__ void qk_step(uint32_t d_tmem, uint64_t qd, uint64_t kd, uint32_t idesc) {
+  constexpr uint32_t off = ((kk >> 2) * kPanelBytes + (kk & 3) * 32) >> 4;
+  mma_f16_ss_off<off, off>(d_tmem, qd, kd, idesc, kk > 0 ? 1u : 0u);
+}
+
+__device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_s, uint32_t k_s) {
+  const uint32_t idesc = idesc_f16_f32(kBlockM, kBlockN, false, false);
+  const uint64_t qd = smem_desc_sw128(q_s, 16, 1024);
+  const uint64_t kd = smem_desc_sw128(k_s, 16, 1024);
+  qk_step<0>(d_tmem, qd, kd, idesc);
+  qk_step<1>(d_tmem, qd, kd, idesc);
+  qk_step<2>(d_tmem, qd, kd, idesc);
+  qk_step<3>(d_tmem, qd, kd, idesc);
+  qk_step<4>(d_tmem, qd, kd, idesc);
+  qk_step<5>(d_tmem, qd, kd, idesc);
+  qk_step<6>(d_tmem, qd, kd, idesc);
+  qk_step<7>(d_tmem, qd, kd, idesc);
+}
+
+// O_X (+)= P V: A = P from TMEM (8 columns = 16 keys per MMA), B = V, an
+// MN-major operand (16 keys = two 8-row groups of 1 KiB; the two 64-column
+// halves of D are a panel apart).
+template <int kk>
+__device__ __forceinline__ void pv_step(uint32_t o_tmem, uint32_t p_tmem, uint64_t vd,
+                                        uint32_t idesc, uint32_t acc) {
+  constexpr uint32_t a_off = kk * 8;            // TMEM columns
+  constexpr uint32_t b_off = (kk * 2048) / 16;   // 16 keys of V, in 16-byte units
+  mma_f16_ts_off<a_off, b_off>(o_tmem, p_tmem, vd, idesc, (acc || kk > 0) ? 1u : 0u);
+}
+
+__device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint32_t v_s,
+                                         bool accumulate) {
+  const uint32_t idesc = idesc_f16_f32(kBlockM, kHeadDim, false, true);
+  const uint64_t vd = smem_desc_sw128(v_s, kPanelBytes, 1024);
+  const uint32_t acc = accumulate ? 1u : 0u;
+  pv_step<0>(o_tmem, p_tmem, vd, idesc, acc);
+  pv_step<1>(o_tmem, p_tmem, vd, idesc, acc);
+  pv_step<2>(o_tmem, p_tmem, vd, idesc, acc);
+  pv_step<3>(o_tmem, p_tmem, vd, idesc, acc);
+  pv_step<4>(o_tmem, p_tmem, vd, idesc, acc);
+  pv_step<5>(o_tmem, p_tmem, vd, idesc, acc);
+  pv_step<6>(o_tmem, p_tmem, vd, idesc, acc);
+  pv_step<7>(o_tmem, p_tmem, vd, idesc, acc);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
   extern __shared__ uint8_t smem_raw[];
-  Smem* sm = reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                     ~static_cast<uintptr_t>(1023));
+  SharedFwd* sm = reinterpret_cast<SharedFwd*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~static_cast<uintptr_t>(1023));
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-
-  const int n_qb = p.S / kBlockM;
-  const int qb = n_qb - 1 - static_cast<int>(blockIdx.x);  // heaviest causal tiles first
-  const int hq = blockIdx.y;
-  const int b = blockIdx.z;
-  const int g = hq / (p.Hq / p.Hkv);
-  const int n_kv = p.causal ? qb + 1 : n_qb;
-  const int q_row0 = (b * p.Hq + hq) * p.S + qb * kBlockM;
-  const int kv_row0 = (b * p.Hkv + g) * p.S;
   const uint64_t to = p.timeout_ns;
 
   if (threadIdx.x == 0) {
+    sm->n_listed = (p.mode == 1) ? *reinterpret_cast<volatile unsigned int*>(p.redo) : 0u;
     mbar_init(smem_addr(&sm->q_full), 1);
+    mbar_init(smem_addr(&sm->q_empty), 1);
     for (int s = 0; s < kStages; ++s) {
       mbar_init(smem_addr(&sm->k_full[s]), 1);
       mbar_init(smem_addr(&sm->v_full[s]), 1);
       mbar_init(smem_addr(&sm->kv_empty[s]), 1);
     }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(smem_addr(&sm->s_full[s]), 1);
-      mbar_init(smem_addr(&sm->p_full[s]), kBlockM);
-      mbar_init(smem_addr(&sm->pv_done[s]), 1);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(smem_addr(&sm->s_full[x]), 1);
+      mbar_init(smem_addr(&sm->p_full[x]), kBlockM);
+      mbar_init(smem_addr(&sm->o_done[x]), 1);
+      mbar_init(smem_addr(&sm->o_free[x]), kBlockM);
+      mbar_init(smem_addr(&sm->stats_ready[x]), kBlockM);
     }
     mbar_init(smem_addr(&sm->drain), 1);
     sm->abort = 0;
+    sm->item_flag[0] = sm->item_flag[1] = 0;
+    sm->item_warps[0] = sm->item_warps[1] = 0;
     fence_mbar_init();
   }
-  if (warp == 4 && lane == 0) {
-    tma_prefetch_desc(&tm_q);
-    tma_prefetch_desc(&tm_k);
-    tma_prefetch_desc(&tm_v);
-  }
-  if (warp == 5) {
-    tmem_alloc(smem_addr(&sm->tmem_base), kTmemCols);
-    tmem_relinquish();
-  }
-  tc_fence_before();
   __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = sm->tmem_base;
-  volatile int* abort = &sm->abort;
+  const unsigned int n_listed = sm->n_listed;
+  const bool has_work = work_item(p, 0, n_listed) >= 0;
 
-  if (warp == 4) {
-    // ---------------------------------------------------------------- producer
-    if (lane == 0) {
-      const uint32_t q_s = smem_addr(sm->q);
-      mbar_arrive_expect_tx(smem_addr(&sm->q_full), kTileBytes);
-      tma_load_2d(q_s, &tm_q, smem_addr(&sm->q_full), 0, q_row0);
-      tma_load_2d(q_s + kPanelBytes, &tm_q, smem_addr(&sm->q_full), 64, q_row0);
-      int j = 0;
-      for (; j < n_kv; ++j) {
-        const int st = j % kStages;
-        const int rnd = j / kStages;
-        if (rnd > 0 &&
-            !mbar_wait(smem_addr(&sm->kv_empty[st]), (rnd - 1) & 1, abort, to, kSiteProducerEmpty))
-          break;
-        const int row = kv_row0 + j * kBlockN;
-        const uint32_t kf = smem_addr(&sm->k_full[st]);
-        const uint32_t vf = smem_addr(&sm->v_full[st]);
-        const uint32_t k_s = smem_addr(sm->k[st]);
-        const uint32_t v_s = smem_addr(sm->v[st]);
-        mbar_arrive_expect_tx(kf, kTileBytes);
-        tma_load_2d(k_s, &tm_k, kf, 0, row);
-        tma_load_2d(k_s + kPanelBytes, &tm_k, kf, 64, row);
-        mbar_arrive_expect_tx(vf, kTileBytes);
-        tma_load_2d(v_s, &tm_v, vf, 0, row);
-        tma_load_2d(v_s + kPanelBytes, &tm_v, vf, 64, row);
-      }
-      if (*abort) {
-        // let every copy still in flight land before the CTA exits
-        drain_wait(smem_addr(&sm->q_full), 0, to);
-        for (int t = (j > kStages ? j - kStages : 0); t < j; ++t) {
-          drain_wait(smem_addr(&sm->k_full[t % kStages]), (t / kStages) & 1, to);
-          drain_wait(smem_addr(&sm->v_full[t % kStages]), (t / kStages) & 1, to);
-        }
-      }
+  if (has_work) {
+    if (warp == kMmaWarp) {
+      tmem_alloc(smem_addr(&sm->tmem_base), kTmemCols);
+      tmem_relinquish();
     }
-  } else if (warp == 5) {
-    // ---------------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc_qk = idesc_f16_f32(kBlockM, kBlockN, false, false);
-      constexpr uint32_t idesc_pv = idesc_f16_f32(kBlockM, kHeadDim, false, true);
-      const uint32_t q_s = smem_addr(sm->q);
-      // O += P_t V_t; returns false if a wait ran out
-      auto issue_pv = [&](int t) -> bool {
-        const int pb = t & 1;
-        const int st = t % kStages;
-        if (!mbar_wait(smem_addr(&sm->p_full[pb]), (t >> 1) & 1, abort, to, kSiteMmaP)) return false;
-        if (!mbar_wait(smem_addr(&sm->v_full[st]), (t / kStages) & 1, abort, to, kSiteMmaV))
-          return false;
-        tc_fence_after();
-        const uint32_t v_s = smem_addr(sm->v[st]);
-#pragma unroll
-        for (int kk = 0; kk < kBlockN / 16; ++kk) {
-          // V is MN-major: 16 keys = two 8-row groups of 1 KiB; the two
-          // 64-column panels of D are kPanelBytes apart.
-          const uint64_t bdesc = smem_desc_sw128(v_s + kk * 2048, kPanelBytes, 1024);
-          mma_f16_ts(tmem + kTmemO, tmem + pb * 128 + kk * 8, bdesc, idesc_pv,
-                     (t > 0 || kk > 0) ? 1u : 0u);
-        }
-        tc_commit(smem_addr(&sm->kv_empty[st]));
-        tc_commit(smem_addr(&sm->pv_done[pb]));
-        return true;
-      };
-      bool ok = mbar_wait(smem_addr(&sm->q_full), 0, abort, to, kSiteMmaQ);
-      for (int j = 0; ok && j < n_kv; ++j) {
-        const int st = j % kStages;
-        if (!mbar_wait(smem_addr(&sm->k_full[st]), (j / kStages) & 1, abort, to, kSiteMmaK)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t k_s = smem_addr(sm->k[st]);
-#pragma unroll
-        for (int kk = 0; kk < kHeadDim / 16; ++kk) {
-          // K-major: 16 columns = 32 bytes inside a 128-byte swizzled row;
-          // columns 64..127 live in the second panel.
-          const uint32_t off = (kk >> 2) * kPanelBytes + (kk & 3) * 32;
-          mma_f16_ss(tmem + (j & 1) * 128, smem_desc_sw128(q_s + off, 16, 1024),
-                     smem_desc_sw128(k_s + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
-        }
-        tc_commit(smem_addr(&sm->s_full[j & 1]));
-        if (j > 0 && !issue_pv(j - 1)) ok = false;
-      }
-      if (ok) issue_pv(n_kv - 1);
-      // every MMA issued must complete before TMEM is released
-      tc_commit(smem_addr(&sm->drain));
-      drain_wait(smem_addr(&sm->drain), 0, to);
+    if (warp == kProducerWarp && lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
     }
-    __syncwarp();
-  } else {
-    // ---------------------------------------------------------------- softmax
-    const int r = threadIdx.x;  // query row inside the tile == TMEM lane
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-    const float sc = p.scale_log2;
-    float m_use = -INFINITY;  // reference max (log2 units) shared by O and l
-    float l = 0.f;
-    bool ok = true;
-    for (int j = 0; j < n_kv; ++j) {
-      const int sb = j & 1;
-      // tcgen05.ld/st are warp-collective: every wait outcome is made
-      // warp-uniform before the warp touches TMEM.
-      ok = mbar_wait(smem_addr(&sm->s_full[sb]), (j >> 1) & 1, abort, to, kSiteSoftmaxS);
-      if (!__all_sync(0xffffffffu, ok)) {
-        ok = false;
-        break;
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm->tmem_base;
+    volatile int* abort = &sm->abort;
+
+    if (warp >= kProducerWarp) {
+      regs_dec<kRegsOther>();
+      if (warp == kProducerWarp && lane == 0) {
+        // ------------------------------------------------------------ producer
+        const uint64_t keep = l2_policy_evict_last();     // K/V: reused by many items
+        const uint64_t once = l2_policy_evict_first();    // Q: read once
+        int rc = 0;
+        int k = 0;
+        int item;
+        bool ok = true;
+        for (; ok && (item = work_item(p, k, n_listed)) >= 0; ++k) {
+          const Item it = decode_item(p, item);
+          if (k > 0 && !mbar_wait(smem_addr(&sm->q_empty), (k - 1) & 1, abort, to, kSiteProducerQ)) {
+            ok = false;
+            break;
+          }
+          const int q_row = (it.b * p.Hq + it.hq) * p.S + it.qb2 * kItemRows;
+          const uint32_t qf = smem_addr(&sm->q_full);
+          mbar_arrive_expect_tx(qf, 2 * kTileBytes);
+#pragma unroll
+          for (int x = 0; x < 2; ++x) {
+            const uint32_t q_s = smem_addr(sm->q[x]);
+            tma_load_2d_hint(q_s, &tm_q, qf, 0, q_row + x * kBlockM, once);
+            tma_load_2d_hint(q_s + kPanelBytes, &tm_q, qf, 64, q_row + x * kBlockM, once);
+          }
+          const int kv_row = (it.b * p.Hkv + it.g) * p.S;
+          for (int j = 0; j < it.n_blocks; ++j, ++rc) {
+            const int st = rc % kStages;
+            if (rc >= kStages && !mbar_wait(smem_addr(&sm->kv_empty[st]), ring_parity(rc) ^ 1, abort,
+                                            to, kSiteProducerKV)) {
+              ok = false;
+              break;
+            }
+            const uint32_t kf = smem_addr(&sm->k_full[st]);
+            const uint32_t vf = smem_addr(&sm->v_full[st]);
+            const uint32_t k_s = smem_addr(sm->k[st]);
+            const uint32_t v_s = smem_addr(sm->v[st]);
+            mbar_arrive_expect_tx(kf, kTileBytes);
+            tma_load_2d_hint(k_s, &tm_k, kf, 0, kv_row + j * kBlockN, keep);
+            tma_load_2d_hint(k_s + kPanelBytes, &tm_k, kf, 64, kv_row + j * kBlockN, keep);
+            mbar_arrive_expect_tx(vf, kTileBytes);
+            tma_load_2d_hint(v_s, &tm_v, vf, 0, kv_row + j * kBlockN, keep);
+            tma_load_2d_hint(v_s + kPanelBytes, &tm_v, vf, 64, kv_row + j * kBlockN, keep);
+          }
+        }
+        if (*abort) {
+          // every copy still in flight must land before the CTA exits: the
+          // last Q load and the last load of each ring stage
+          if (k > 0) drain_wait(smem_addr(&sm->q_full), (k - 1) & 1, to);
+          for (int t = (rc > kStages ? rc - kStages : 0); t < rc; ++t) {
+            drain_wait(smem_addr(&sm->k_full[t % kStages]), ring_parity(t), to);
+            drain_wait(smem_addr(&sm->v_full[t % kStages]), ring_parity(t), to);
+          }
+        }
+      } else if (warp == kMmaWarp && lane == 0) {
+        // ------------------------------------------------------------ MMA issuer
+        const bool hilo = p.mode == 1;
+        int rc = 0;
+        int pcnt[2] = {0, 0};
+        int acnt[2] = {0, 0};  // items so far in which tile X was active
+        bool ok = true;
+        int item;
+        for (int k = 0; ok && (item = work_item(p, k, n_listed)) >= 0; ++k) {
+          const Item it = decode_item(p, item);
+          const int n_b = it.n_blocks;
+          if (!mbar_wait(smem_addr(&sm->q_full), k & 1, abort, to, kSiteMmaQ)) {
+            ok = false;
+            break;
+          }
+          for (int j = 0; ok && j <= n_b; ++j) {
+            const int st_k = (rc + j) % kStages;
+            const int st_v = (rc + j + kStages - 1) % kStages;
+            if (j < n_b &&
+                !mbar_wait(smem_addr(&sm->k_full[st_k]), ring_parity(rc + j), abort, to, kSiteMmaK)) {
+              ok = false;
+              break;
+            }
+            if (j >= 1 && !mbar_wait(smem_addr(&sm->v_full[st_v]), ring_parity(rc + j - 1), abort,
+                                     to, kSiteMmaV)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            for (int x = 0; ok && x < 2; ++x) {
+              const int n_x = it.n_kv[x];
+              if (j >= 1 && j - 1 < n_x) {
+                // the epilogue must have read O_X of the tile's previous item
+                if (j == 1 && acnt[x] > 0 &&
+                    !mbar_wait(smem_addr(&sm->o_free[x]), (acnt[x] - 1) & 1, abort, to, kSiteMmaO)) {
+                  ok = false;
+                  break;
+                }
+                if (!mbar_wait(smem_addr(&sm->p_full[x]), pcnt[x] & 1, abort, to, kSiteMmaP)) {
+                  ok = false;
+                  break;
+                }
+                ++pcnt[x];
+                tc_fence_after();
+                const uint32_t v_s = smem_addr(sm->v[st_v]);
+                issue_pv(tmem + tmem_o_col(x), tmem + tmem_s_col(x), v_s, j - 1 > 0);
+                if (hilo) issue_pv(tmem + tmem_o_col(x), tmem + tmem_s_col(x) + 64, v_s, true);
+                if (j == n_x) tc_commit(smem_addr(&sm->o_done[x]));
+              }
+              if (j < n_x) {
+                issue_qk(tmem + tmem_s_col(x), smem_addr(sm->q[x]), smem_addr(sm->k[st_k]));
+                tc_commit(smem_addr(&sm->s_full[x]));
+              }
+            }
+            if (ok && j == n_b - 1) tc_commit(smem_addr(&sm->q_empty));  // last S issued
+            if (ok && j >= 1) tc_commit(smem_addr(&sm->kv_empty[st_v]));
+          }
+          rc += n_b;
+          acnt[0] += it.n_kv[0] > 0;
+          acnt[1] += it.n_kv[1] > 0;
+        }
+        // every MMA issued must complete before TMEM is released
+        tc_commit(smem_addr(&sm->drain));
+        drain_wait(smem_addr(&sm->drain), 0, to);
       }
-      tc_fence_after();
-      const uint32_t s_t = lane_base + sb * 128;
-      uint32_t u[4][32];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(s_t + c * 32, u[c]);
-      tmem_wait_ld();
-      float sv[128];
-#pragma unroll
-      for (int c = 0; c < 4; ++c)
-#pragma unroll
-        for (int i = 0; i < 32; ++i) sv[c * 32 + i] = __uint_as_float(u[c][i]);
-      if (p.causal && j == qb) {
-#pragma unroll
-        for (int c = 0; c < 128; ++c)
-          if (c > r) sv[c] = -INFINITY;
-      }
-      float mx = sv[0];
-#pragma unroll
-      for (int c = 1; c < 128; ++c) mx = fmaxf(mx, sv[c]);
-      const float cand = mx * sc;
-      if (j == 0) {
-        m_use = cand;
-      } else {
-        const bool grow = cand > m_use + kRescaleLog2;
-        if (__any_sync(0xffffffffu, grow)) {
-          const float alpha = grow ? ex2_approx(m_use - cand) : 1.0f;
-          // O must already hold P_{j-1} V_{j-1} before it is rescaled
-          ok = mbar_wait(smem_addr(&sm->pv_done[(j - 1) & 1]), ((j - 1) >> 1) & 1, abort, to,
-                         kSiteSoftmaxO);
+      __syncwarp();
+    } else if (warp >= kEpilogueWarp0) {
+      // -------------------------------------------------------------- epilogue
+      regs_dec<kRegsEpilogue>();
+      const int r = (warp - kEpilogueWarp0) * 32 + lane;
+      const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+      int acnt[2] = {0, 0};  // items so far in which tile X was active
+      int item;
+      for (int k = 0; (item = work_item(p, k, n_listed)) >= 0; ++k) {
+        const Item it = decode_item(p, item);
+        bool flag = false;
+        bool ok = true;
+#pragma unroll 1
+        for (int x = 0; x < 2; ++x) {
+          if (it.n_kv[x] == 0) continue;
+          const int a = acnt[x]++;
+          ok = mbar_wait(smem_addr(&sm->o_done[x]), a & 1, abort, to, kSiteEpilogueO) &&
+               mbar_wait(smem_addr(&sm->stats_ready[x]), a & 1, abort, to, kSiteEpilogueStats);
           if (!__all_sync(0xffffffffu, ok)) {
             ok = false;
             break;
           }
           tc_fence_after();
+          const float m_use = sm->stat_m[a & 1][x][r];
+          const float l = sm->stat_l[a & 1][x][r];
+          const float inv_l = 1.0f / l;
+          const int row = (it.b * p.Hq + it.hq) * p.S + it.qb2 * kItemRows + x * kBlockM + r;
+          uint4* orow = reinterpret_cast<uint4*>(p.o + static_cast<size_t>(row) * kHeadDim);
+          float omax = 0.f;
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t w[32];
-            tmem_ld32(lane_base + kTmemO + c * 32, w);
+          for (int c = 0; c < 8; ++c) {
+            uint32_t w[16];
+            tmem_ld16(lane_base + tmem_o_col(x) + c * 16, w);
             tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(__uint_as_float(w[i]) * alpha);
-            tmem_st32(lane_base + kTmemO + c * 32, w);
+            for (int v4 = 0; v4 < 2; ++v4) {
+              float f[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                f[e] = __uint_as_float(w[v4 * 8 + e]) * inv_l;
+                omax = fmaxf(omax, fabsf(f[e]));
+              }
+              uint4 pk;
+              pk.x = pack_half2(f[0], f[1]);
+              pk.y = pack_half2(f[2], f[3]);
+              pk.z = pack_half2(f[4], f[5]);
+              pk.w = pack_half2(f[6], f[7]);
+              orow[c * 2 + v4] = pk;
+            }
           }
-          if (grow) {
-            l *= alpha;
-            m_use = cand;
+          tc_fence_before();
+          mbar_arrive(smem_addr(&sm->o_free[x]));
+          p.lse[row] = (m_use + log2f(l)) * kLn2;
+          flag |= omax >= kRedoThreshold;
+        }
+        if (!ok) break;
+        if (p.mode == 0) {
+          // One redo-list entry per item if any of its rows needs it.  The
+          // last of the four epilogue warps to finish the item appends it (no
+          // barrier, so a warp that gave up on a wait cannot block the
+          // others).  Slots are per item parity: a warp reaches item k+2 only
+          // after every warp has finished item k.
+          const bool any = __any_sync(0xffffffffu, flag);
+          if (lane == 0) {
+            if (any) atomicOr(&sm->item_flag[k & 1], 1);
+            __threadfence_block();
+            if (atomicAdd(&sm->item_warps[k & 1], 1) == 3) {
+              if (atomicExch(&sm->item_flag[k & 1], 0)) {
+                const unsigned int slot = atomicAdd(p.redo, 1u);
+                if (slot < p.redo_capacity)
+                  p.redo[kRedoHeaderWords + slot] = static_cast<unsigned int>(item);
+              }
+              sm->item_warps[k & 1] = 0;
+            }
           }
         }
       }
-      const float neg_m = -m_use;
+    } else {
+      // -------------------------------------------------------------- softmax
+      regs_inc<kRegsSoftmax>();
+      const int x = warp >> 2;  // tile
+      const int r = (warp & 3) * 32 + lane;
+      const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+      const uint32_t s_t = lane_base + tmem_s_col(x);
+      const uint32_t o_t = lane_base + tmem_o_col(x);
+      const float sc = p.scale_log2;
+      const bool hilo = p.mode == 1;
+      int scnt = 0;
+      int acnt = 0;  // items so far in which this tile was active
+      int item;
+      for (int k = 0; (item = work_item(p, k, n_listed)) >= 0; ++k) {
+        const Item it = decode_item(p, item);
+        const int n_x = it.n_kv[x];
+        if (n_x == 0) continue;
+        const int diag = p.causal ? n_x - 1 : -1;
+        float m_use = -INFINITY;
+        float l = 0.f;
+        bool ok = true;
+        for (int j = 0; j < n_x; ++j, ++scnt) {
+          ok = mbar_wait(smem_addr(&sm->s_full[x]), scnt & 1, abort, to, kSiteSoftmaxS);
+          if (!__all_sync(0xffffffffu, ok)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          // the row of S_X in 128 registers (fp32 bits)
+          uint32_t u[128];
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        uint32_t ph[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float p0 = ex2_approx(fmaf(sv[c * 64 + 2 * i], sc, neg_m));
-          const float p1 = ex2_approx(fmaf(sv[c * 64 + 2 * i + 1], sc, neg_m));
-          l += p0 + p1;
-          ph[i] = pack_half2(p0, p1);
-        }
-        tmem_st32(s_t + c * 32, ph);
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(smem_addr(&sm->p_full[sb]));
-    }
-    if (ok) {
-      const int t = n_kv - 1;
-      ok = mbar_wait(smem_addr(&sm->pv_done[t & 1]), (t >> 1) & 1, abort, to, kSiteEpilogueO);
-      if (__all_sync(0xffffffffu, ok)) {
-        tc_fence_after();
-        const float inv_l = 1.0f / l;
-        uint4* orow = reinterpret_cast<uint4*>(p.o + static_cast<size_t>(q_row0 + r) * kHeadDim);
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t w[32];
-          tmem_ld32(lane_base + kTmemO + c * 32, w);
+          for (int c = 0; c < 4; ++c)
+            tmem_ld32(s_t + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&u[c * 32]));
           tmem_wait_ld();
+          if (j == diag) {
 #pragma unroll
-          for (int v4 = 0; v4 < 4; ++v4) {
-            uint4 pk;
-            pk.x = pack_half2(__uint_as_float(w[v4 * 8 + 0]) * inv_l,
-                              __uint_as_float(w[v4 * 8 + 1]) * inv_l);
-            pk.y = pack_half2(__uint_as_float(w[v4 * 8 + 2]) * inv_l,
-                              __uint_as_float(w[v4 * 8 + 3]) * inv_l);
-            pk.z = pack_half2(__uint_as_float(w[v4 * 8 + 4]) * inv_l,
-                              __uint_as_float(w[v4 * 8 + 5]) * inv_l);
-            pk.w = pack_half2(__uint_as_float(w[v4 * 8 + 6]) * inv_l,
-                              __uint_as_float(w[v4 * 8 + 7]) * inv_l);
-            orow[c * 4 + v4] = pk;
+            for (int c = 0; c < 128; ++c)
+              if (c > r) u[c] = 0xff800000u;  // -inf
           }
+          float mx8[8];
+#pragma unroll
+          for (int t = 0; t < 8; ++t) mx8[t] = __uint_as_float(u[t]);
+#pragma unroll
+          for (int c = 8; c < 128; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(u[c]));
+#pragma unroll
+          for (int t = 0; t < 4; ++t) mx8[t] = fmaxf(mx8[t], mx8[t + 4]);
+          const float cand = fmaxf(fmaxf(mx8[0], mx8[2]), fmaxf(mx8[1], mx8[3])) * sc;
+          if (j == 0) {
+            m_use = cand;
+          } else {
+            const bool grow = cand > m_use + kRescaleLog2;
+            if (__any_sync(0xffffffffu, grow)) {
+              // O_X holds P(j-1) V_{j-1} already (it completed before S(j))
+              const float alpha = grow ? ex2_approx(m_use - cand) : 1.0f;
+#pragma unroll 1
+              for (int c = 0; c < 4; ++c) {
+                uint32_t w[32];
+                tmem_ld32(o_t + c * 32, w);
+                tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(__uint_as_float(w[i]) * alpha);
+                tmem_st32(o_t + c * 32, w);
+              }
+              if (grow) {
+                l *= alpha;
+                m_use = cand;
+              }
+            }
+          }
+          const float neg_m = -m_use;
+          float lp[4] = {0.f, 0.f, 0.f, 0.f};
+          if (!hilo) {
+            // P rounded to fp16; l sums exactly the rounded values
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              uint32_t ph[8];
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                const float p0 = ex2_approx(fmaf(__uint_as_float(u[c * 16 + 2 * i]), sc, neg_m));
+                const float p1 = ex2_approx(fmaf(__uint_as_float(u[c * 16 + 2 * i + 1]), sc, neg_m));
+                ph[i] = pack_half2(p0, p1);
+                lp[i & 3] = add_half2_f32(ph[i], lp[i & 3]);
+              }
+              tmem_st8(s_t + c * 8, ph);
+            }
+          } else {
+            // P = hi + lo, both fp16: hi over columns [0,64), lo over [64,128)
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              uint32_t ph[8], pl[8];
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                const float p0 = ex2_approx(fmaf(__uint_as_float(u[c * 16 + 2 * i]), sc, neg_m));
+                const float p1 = ex2_approx(fmaf(__uint_as_float(u[c * 16 + 2 * i + 1]), sc, neg_m));
+                ph[i] = pack_half2(p0, p1);
+                const float2 h = __half22float2(*reinterpret_cast<const __half2*>(&ph[i]));
+                pl[i] = pack_half2(p0 - h.x, p1 - h.y);
+                lp[i & 3] += p0 + p1;
+              }
+              tmem_st8(s_t + c * 8, ph);
+              tmem_st8(s_t + 64 + c * 8, pl);
+            }
+          }
+          l += (lp[0] + lp[1]) + (lp[2] + lp[3]);
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(smem_addr(&sm->p_full[x]));
         }
-        p.lse[q_row0 + r] = (m_use + log2f(l)) * kLn2;
+        if (!ok) break;
+        sm->stat_m[acnt & 1][x][r] = m_use;
+        sm->stat_l[acnt & 1][x][r] = l;
+        ++acnt;
+        mbar_arrive(smem_addr(&sm->stats_ready[x]));
       }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kMmaWarp) {
+      tc_fence_after();
+      tmem_dealloc(tmem, kTmemCols);
     }
   }
 
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 5) {
-    tc_fence_after();
-    tmem_dealloc(tmem, kTmemCols);
+  if (p.mode == 1) {
+    // the last CTA out empties the redo list for the next call on this stream
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      __threadfence();
+      const unsigned int prev = atomicAdd(p.redo + 1, 1u);
+      if (prev == gridDim.x - 1) {
+        p.redo[0] = 0;
+        p.redo[1] = 0;
+        __threadfence();
+      }
+    }
   }
 }
 
