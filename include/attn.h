@@ -24,8 +24,12 @@
  *   - Layouts are dense row-major: Q, O [B, Hq, S, D]; K, V [B, Hkv, S, D];
  *     LSE [B, Hq, S].  "Device" pointers are CUDA device (or managed)
  *     addresses on the current device; "host" pointers are CPU addresses.
- *   - The caller owns every buffer.  The library never allocates device or
- *     host memory in these calls and keeps no pointer after returning.
+ *   - The caller owns every input and output buffer; the library keeps no
+ *     pointer to them after returning.  Besides those, attn_fwd (and
+ *     attn_fwd_host, which calls it) needs a small device scratch list: the
+ *     first call for each (device, stream) pair allocates it with cudaMalloc
+ *     (256 KiB + 16 B) and zeroes it on that stream; it is kept for later
+ *     calls on that pair until the process exits.  Nothing else allocates.
  *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls
  *     are asynchronous with respect to the host unless stated otherwise.
  *   - Arguments are validated before anything is launched; a rejected call
@@ -65,8 +69,12 @@ typedef enum attn_status {
  *   B, Hq, Hkv, S, D: sizes; Hq % Hkv == 0; D == 128; S % 128 == 0.
  *   causal: nonzero for the causal mask j <= i (square, Sq == Sk == S).
  *   stream: cudaStream_t to launch on.
- * Returns ATTN_OK once the kernel is enqueued; errors as listed above.  The
- * outputs must not overlap the inputs.
+ * Returns ATTN_OK once the kernels are enqueued; errors as listed above.  The
+ * outputs must not overlap the inputs.  Two kernels run on `stream`: the
+ * fused pass over every 256-row work item, then a pass that recomputes, with
+ * probabilities split into two fp16 parts, only the items the first pass
+ * listed (those with a row max|O| >= 3.98, where fp16 output rounding leaves
+ * almost no error budget); it exits at once when the list is empty.
  */
 attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
                      int B, int Hq, int Hkv, int S, int D, int causal, void* stream);
