@@ -17,9 +17,10 @@ LIB_PATH = os.path.join(_PKG, "libattn_b200.so")
 
 ATTN_OK = 0
 ATTN_ERR_DEVICE_TIMEOUT = 6
+ATTN_ERR_TOO_LARGE = 8
 STATUS_NAMES = {0: "ATTN_OK", 1: "ATTN_ERR_NULL", 2: "ATTN_ERR_SHAPE", 3: "ATTN_ERR_ALIGN",
                 4: "ATTN_ERR_UNSUPPORTED", 5: "ATTN_ERR_CUDA", 6: "ATTN_ERR_DEVICE_TIMEOUT",
-                7: "ATTN_ERR_WORKSPACE"}
+                7: "ATTN_ERR_WORKSPACE", 8: "ATTN_ERR_TOO_LARGE"}
 
 _lib = None
 
@@ -42,6 +43,8 @@ def load() -> ctypes.CDLL:
     vp, i, u64, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_uint64, ctypes.c_size_t
     lib.attn_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, vp]
     lib.attn_fwd.restype = i
+    lib.attn_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, vp]
+    lib.attn_fwd_noalloc.restype = i
     lib.attn_fwd_host.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, vp, sz, vp]
     lib.attn_fwd_host.restype = i
     lib.attn_fwd_host_workspace_bytes.argtypes = [i, i, i, i, i]
@@ -115,6 +118,19 @@ def attn_fwd_raw(q_ptr: int, k_ptr: int, v_ptr: int, o_ptr: int, lse_ptr: int, B
     """The C entry point with raw addresses; returns the status code."""
     return int(load().attn_fwd(q_ptr, k_ptr, v_ptr, o_ptr, lse_ptr, B, Hq, Hkv, S, D,
                                int(bool(causal)), stream_ptr))
+
+
+def attn_fwd_noalloc_raw(q_ptr: int, k_ptr: int, v_ptr: int, o_ptr: int, lse_ptr: int, B: int,
+                        Hq: int, Hkv: int, S: int, D: int, causal: bool, stream_ptr: int) -> int:
+    """The no-allocation C entry point with raw addresses; returns the status
+    code.  For callers that cannot let the library call cudaMalloc (memory
+    planned up front, their own caching allocator, or no tolerance for the
+    device synchronization an allocation may cause): its scratch is a fixed
+    array inside the library, so sizes above B*Hq*ceil(S/256) = 131072 work
+    items are rejected, and calls that overlap on the GPU must not share a
+    device."""
+    return int(load().attn_fwd_noalloc(q_ptr, k_ptr, v_ptr, o_ptr, lse_ptr, B, Hq, Hkv, S, D,
+                                       int(bool(causal)), stream_ptr))
 
 
 def host_workspace_bytes(B: int, Hq: int, Hkv: int, S: int, D: int) -> int:

@@ -154,6 +154,9 @@ const char* attn_status_string(attn_status s) {
     case ATTN_ERR_CUDA: return "ATTN_ERR_CUDA: a CUDA call failed";
     case ATTN_ERR_DEVICE_TIMEOUT: return "ATTN_ERR_DEVICE_TIMEOUT: a kernel wait ran out";
     case ATTN_ERR_WORKSPACE: return "ATTN_ERR_WORKSPACE: device workspace too small";
+    case ATTN_ERR_TOO_LARGE:
+      return "ATTN_ERR_TOO_LARGE: B*Hq*ceil(S/256) exceeds attn_fwd_noalloc's fixed scratch "
+             "(131072 work items)";
   }
   return "ATTN_ERR_UNKNOWN";
 }
@@ -288,4 +291,91 @@ extern "C" attn_status attn_selftest_wait_timeout(uint64_t timeout_ns, void* str
   selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(timeout_ns);
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
   return attn_device_status(stream, nullptr);
+}
+
+// ---------------------------------------------------------------------------
+// attn_fwd_noalloc: the same two launches as attn_fwd, with the redo list in
+// a fixed array of this file instead of memory from cudaMalloc.
+// ---------------------------------------------------------------------------
+namespace attn_b200 {
+namespace {
+
+constexpr unsigned int kNoAllocMaxItems = 1u << 17;  // 131072 items: 512 KiB of ids
+
+// Header {count, done, -, -} then up to kNoAllocMaxItems item ids.  Every
+// device that loads the library holds one copy until the process exits.
+static __device__ __align__(256) unsigned int g_noalloc_redo[kRedoHeaderWords + kNoAllocMaxItems];
+
+// Device address of g_noalloc_redo, looked up once per device with that
+// device current (host code cannot use the symbol itself as an address).
+unsigned int* g_noalloc_ptr[kMaxDevices];
+std::mutex g_noalloc_mutex;
+
+unsigned int* noalloc_scratch(int dev) {
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (!g_noalloc_ptr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_redo) != cudaSuccess || !ptr) return nullptr;
+    g_noalloc_ptr[dev] = static_cast<unsigned int*>(ptr);
+  }
+  return g_noalloc_ptr[dev];
+}
+
+}  // namespace
+}  // namespace attn_b200
+
+extern "C" attn_status attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o,
+                                        float* lse, int B, int Hq, int Hkv, int S, int D,
+                                        int causal, void* stream) {
+  if (!q || !k || !v || !o || !lse) return ATTN_ERR_NULL;
+  attn_status st = validate_sizes(B, Hq, Hkv, S, D);
+  if (st != ATTN_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+    return ATTN_ERR_ALIGN;
+  const int n_qb = S / kBlockM;
+  const int n_qb2 = (n_qb + 1) / 2;
+  const long long n_items = static_cast<long long>(B) * Hq * n_qb2;
+  if (n_items > kNoAllocMaxItems) return ATTN_ERR_TOO_LARGE;
+  int dev = 0;
+  st = device_setup(&dev);
+  if (st != ATTN_OK) return st;
+  unsigned int* scratch = noalloc_scratch(dev);
+  if (!scratch) return ATTN_ERR_CUDA;
+
+  CUtensorMap tm_q, tm_k, tm_v;
+  if (!encode_rows_map(&tm_q, q, static_cast<uint64_t>(B) * Hq * S) ||
+      !encode_rows_map(&tm_k, k, static_cast<uint64_t>(B) * Hkv * S) ||
+      !encode_rows_map(&tm_v, v, static_cast<uint64_t>(B) * Hkv * S))
+    return ATTN_ERR_CUDA;
+
+  FwdParams p;
+  p.o = static_cast<__half*>(o);
+  p.lse = lse;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.S = S;
+  p.causal = causal ? 1 : 0;
+  p.n_qb = n_qb;
+  p.n_qb2 = n_qb2;
+  p.group = Hq / Hkv;
+  p.n_items = static_cast<int>(n_items);
+  p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
+  p.timeout_ns = g_timeout_ns.load();
+  p.redo = scratch;
+  p.redo_capacity = kNoAllocMaxItems;  // >= n_items: the list cannot overflow
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+
+  // the shared array keeps the previous call's header: start from an empty list
+  if (cudaMemsetAsync(scratch, 0, kRedoHeaderWords * sizeof(unsigned int), cs) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  const int sms = g_dev_sms[dev];
+  p.mode = 0;
+  attn_fwd_kernel<<<p.n_items < sms ? p.n_items : sms, kThreads, fwd_smem_bytes(), cs>>>(tm_q, tm_k,
+                                                                                       tm_v, p);
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  p.mode = 1;
+  attn_fwd_kernel<<<sms, kThreads, fwd_smem_bytes(), cs>>>(tm_q, tm_k, tm_v, p);
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  return ATTN_OK;
 }

@@ -57,7 +57,8 @@ typedef enum attn_status {
   ATTN_ERR_UNSUPPORTED = 4,    /* D != 128, S % 128 != 0, or not an sm_100 device */
   ATTN_ERR_CUDA = 5,           /* a CUDA runtime / driver call failed */
   ATTN_ERR_DEVICE_TIMEOUT = 6, /* a kernel wait ran out; results are invalid */
-  ATTN_ERR_WORKSPACE = 7       /* the device workspace given is too small */
+  ATTN_ERR_WORKSPACE = 7,      /* the device workspace given is too small */
+  ATTN_ERR_TOO_LARGE = 8       /* more work than attn_fwd_noalloc's fixed scratch holds */
 } attn_status;
 
 /*
@@ -126,6 +127,33 @@ uint64_t attn_set_wait_timeout_ns(uint64_t ns);
  * the bound works).  The GPU context stays usable afterwards.
  */
 attn_status attn_selftest_wait_timeout(uint64_t timeout_ns, void* stream);
+
+/*
+ * attn_fwd_noalloc -- attn_fwd for callers that must not allocate device
+ * memory.  No counterpart in the paper: it exists for library users, not for
+ * the method.  attn_fwd keeps a small device scratch list per (device,
+ * stream) and creates it with cudaMalloc on first use; some callers cannot
+ * allow that: serving engines that reserve all device memory up front for
+ * their caches, frameworks whose own caching allocator must see every byte,
+ * or latency-bound loops where cudaMalloc's implicit device synchronization
+ * or a late out-of-memory failure is unacceptable.  This entry point keeps
+ * its scratch in a fixed array inside the library instead (512 KiB + 16 B per
+ * device, reserved when the library is loaded and held until the process
+ * exits), and calls no cudaMalloc, cudaFree or other allocating routine.
+ *   Arguments, layouts, results and errors: as attn_fwd, plus
+ *   ATTN_ERR_TOO_LARGE when B * Hq * ceil(S / 256) > 131072 (the array's
+ *   capacity in 256-row work items; e.g. B=64, Hq=64, S=8192 fits exactly).
+ *   Set-up: the first call on each device looks up the array's device address
+ *   (cudaGetSymbolAddress) with that device current; make that first call
+ *   before capturing work into a stream graph.
+ *   Sharing: every call on a device uses the same array.  Each call clears its
+ *   header on `stream` before launching, so calls ordered on one stream are
+ *   independent; calls that overlap on the GPU (different streams, or
+ *   different host threads without ordering) race on it and may produce wrong
+ *   outputs.
+ */
+attn_status attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, float* lse,
+                             int B, int Hq, int Hkv, int S, int D, int causal, void* stream);
 
 /* Human-readable name of a status code (static storage, never NULL). */
 const char* attn_status_string(attn_status status);
