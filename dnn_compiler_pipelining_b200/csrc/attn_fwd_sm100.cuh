@@ -20,9 +20,14 @@
 //   warps 0-3   softmax of tile A   (one query row per thread = TMEM lane)
 //   warps 4-7   softmax of tile B
 //   warps 8-11  epilogue: O / l -> fp16, LSE, for both tiles
-//   warp 12     TMA producer: Q_A, Q_B per item, K_j / V_j into a ring
+//   warp 12     TMA producer of Q_A, Q_B (per item) and K_j (a ring)
 //   warp 13     MMA issuer (one thread): S_X = Q_X K_j^T, O_X += P_X V_j
-//   warps 14-15 idle
+//   warp 14     TMA producer of V_j (its own ring)
+//   warp 15     idle
+//
+// K_j and V_j have separate rings and are released separately, each as soon
+// as the last MMA reading it completes (K after both S(j), V after both
+// PV(j)); a K load is then never held back by the later V release.
 //
 // TMEM (512 columns): S_A [0,128), S_B [128,256), O_A [256,384),
 // O_B [384,512).  P_X (fp16) is written over the first 64 columns of S_X
@@ -62,8 +67,9 @@ constexpr float kRedoThreshold = 3.98f;
 constexpr float kLn2 = 0.69314718055994531f;
 
 constexpr int kEpilogueWarp0 = 8;
-constexpr int kProducerWarp = 12;
+constexpr int kProducerWarp = 12;   // Q and K
 constexpr int kMmaWarp = 13;
+constexpr int kProducerVWarp = 14;  // V
 constexpr int kRegsSoftmax = 192;
 constexpr int kRegsEpilogue = 64;
 constexpr int kRegsOther = 64;
@@ -95,7 +101,8 @@ struct FwdParams {
 
 enum WaitSite : uint32_t {
   kSiteProducerQ = 0x101,
-  kSiteProducerKV = 0x102,
+  kSiteProducerK = 0x102,
+  kSiteProducerV = 0x103,
   kSiteMmaQ = 0x201,
   kSiteMmaK = 0x202,
   kSiteMmaV = 0x203,
@@ -114,7 +121,7 @@ struct alignas(1024) SharedFwd {
   float stat_m[2][2][kBlockM];  // [parity of the tile's active-item count][tile][row]
   float stat_l[2][2][kBlockM];
   uint64_t q_full, q_empty;
-  uint64_t k_full[kStages], v_full[kStages], kv_empty[kStages];
+  uint64_t k_full[kStages], v_full[kStages], k_empty[kStages], v_empty[kStages];
   uint64_t s_full[2], p_full[2], o_done[2], o_free[2], stats_ready[2];
   uint64_t drain;
   uint32_t tmem_base;
@@ -242,7 +249,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < kStages; ++s) {
       mbar_init(smem_addr(&sm->k_full[s]), 1);
       mbar_init(smem_addr(&sm->v_full[s]), 1);
-      mbar_init(smem_addr(&sm->kv_empty[s]), 1);
+      mbar_init(smem_addr(&sm->k_empty[s]), 1);
+      mbar_init(smem_addr(&sm->v_empty[s]), 1);
     }
     for (int x = 0; x < 2; ++x) {
       mbar_init(smem_addr(&sm->s_full[x]), 1);
@@ -279,8 +287,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (warp >= kProducerWarp) {
       regs_dec<kRegsOther>();
-      if (warp == kProducerWarp && lane == 0) {
-        // ------------------------------------------------------------ producer
+      if ((warp == kProducerWarp || warp == kProducerVWarp) && lane == 0) {
+        // ------------------------------------------------------------ producers
+        // warp 12: Q_A, Q_B per item and K_j; warp 14: V_j
+        const bool is_v = warp == kProducerVWarp;
         const uint64_t keep = l2_policy_evict_last();     // K/V: reused by many items
         const uint64_t once = l2_policy_evict_first();    // Q: read once
         int rc = 0;
@@ -289,47 +299,46 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool ok = true;
         for (; ok && (item = work_item(p, k, n_listed)) >= 0; ++k) {
           const Item it = decode_item(p, item);
-          if (k > 0 && !mbar_wait(smem_addr(&sm->q_empty), (k - 1) & 1, abort, to, kSiteProducerQ)) {
-            ok = false;
-            break;
-          }
-          const int q_row = (it.b * p.Hq + it.hq) * p.S + it.qb2 * kItemRows;
-          const uint32_t qf = smem_addr(&sm->q_full);
-          mbar_arrive_expect_tx(qf, 2 * kTileBytes);
+          if (!is_v) {
+            if (k > 0 &&
+                !mbar_wait(smem_addr(&sm->q_empty), (k - 1) & 1, abort, to, kSiteProducerQ)) {
+              ok = false;
+              break;
+            }
+            const int q_row = (it.b * p.Hq + it.hq) * p.S + it.qb2 * kItemRows;
+            const uint32_t qf = smem_addr(&sm->q_full);
+            mbar_arrive_expect_tx(qf, 2 * kTileBytes);
 #pragma unroll
-          for (int x = 0; x < 2; ++x) {
-            const uint32_t q_s = smem_addr(sm->q[x]);
-            tma_load_2d_hint(q_s, &tm_q, qf, 0, q_row + x * kBlockM, once);
-            tma_load_2d_hint(q_s + kPanelBytes, &tm_q, qf, 64, q_row + x * kBlockM, once);
+            for (int x = 0; x < 2; ++x) {
+              const uint32_t q_s = smem_addr(sm->q[x]);
+              tma_load_2d_hint(q_s, &tm_q, qf, 0, q_row + x * kBlockM, once);
+              tma_load_2d_hint(q_s + kPanelBytes, &tm_q, qf, 64, q_row + x * kBlockM, once);
+            }
           }
           const int kv_row = (it.b * p.Hkv + it.g) * p.S;
           for (int j = 0; j < it.n_blocks; ++j, ++rc) {
             const int st = rc % kStages;
-            if (rc >= kStages && !mbar_wait(smem_addr(&sm->kv_empty[st]), ring_parity(rc) ^ 1, abort,
-                                            to, kSiteProducerKV)) {
+            const uint32_t empty = smem_addr(is_v ? &sm->v_empty[st] : &sm->k_empty[st]);
+            if (rc >= kStages && !mbar_wait(empty, ring_parity(rc) ^ 1, abort, to,
+                                            is_v ? kSiteProducerV : kSiteProducerK)) {
               ok = false;
               break;
             }
-            const uint32_t kf = smem_addr(&sm->k_full[st]);
-            const uint32_t vf = smem_addr(&sm->v_full[st]);
-            const uint32_t k_s = smem_addr(sm->k[st]);
-            const uint32_t v_s = smem_addr(sm->v[st]);
-            mbar_arrive_expect_tx(kf, kTileBytes);
-            tma_load_2d_hint(k_s, &tm_k, kf, 0, kv_row + j * kBlockN, keep);
-            tma_load_2d_hint(k_s + kPanelBytes, &tm_k, kf, 64, kv_row + j * kBlockN, keep);
-            mbar_arrive_expect_tx(vf, kTileBytes);
-            tma_load_2d_hint(v_s, &tm_v, vf, 0, kv_row + j * kBlockN, keep);
-            tma_load_2d_hint(v_s + kPanelBytes, &tm_v, vf, 64, kv_row + j * kBlockN, keep);
+            const uint32_t full = smem_addr(is_v ? &sm->v_full[st] : &sm->k_full[st]);
+            const uint32_t dst = smem_addr(is_v ? sm->v[st] : sm->k[st]);
+            const CUtensorMap* map = is_v ? &tm_v : &tm_k;
+            mbar_arrive_expect_tx(full, kTileBytes);
+            tma_load_2d_hint(dst, map, full, 0, kv_row + j * kBlockN, keep);
+            tma_load_2d_hint(dst + kPanelBytes, map, full, 64, kv_row + j * kBlockN, keep);
           }
         }
         if (*abort) {
           // every copy still in flight must land before the CTA exits: the
           // last Q load and the last load of each ring stage
-          if (k > 0) drain_wait(smem_addr(&sm->q_full), (k - 1) & 1, to);
-          for (int t = (rc > kStages ? rc - kStages : 0); t < rc; ++t) {
-            drain_wait(smem_addr(&sm->k_full[t % kStages]), ring_parity(t), to);
-            drain_wait(smem_addr(&sm->v_full[t % kStages]), ring_parity(t), to);
-          }
+          if (!is_v && k > 0) drain_wait(smem_addr(&sm->q_full), (k - 1) & 1, to);
+          for (int t = (rc > kStages ? rc - kStages : 0); t < rc; ++t)
+            drain_wait(smem_addr(is_v ? &sm->v_full[t % kStages] : &sm->k_full[t % kStages]),
+                       ring_parity(t), to);
         }
       } else if (warp == kMmaWarp && lane == 0) {
         // ------------------------------------------------------------ MMA issuer
@@ -385,8 +394,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_commit(smem_addr(&sm->s_full[x]));
               }
             }
-            if (ok && j == n_b - 1) tc_commit(smem_addr(&sm->q_empty));  // last S issued
-            if (ok && j >= 1) tc_commit(smem_addr(&sm->kv_empty[st_v]));
+            if (ok && j < n_b) tc_commit(smem_addr(&sm->k_empty[st_k]));  // every S(j) issued
+            if (ok && j == n_b - 1) tc_commit(smem_addr(&sm->q_empty));   // last S of the item
+            if (ok && j >= 1) tc_commit(smem_addr(&sm->v_empty[st_v]));   // every PV(j-1) issued
           }
           rc += n_b;
           acnt[0] += it.n_kv[0] > 0;
