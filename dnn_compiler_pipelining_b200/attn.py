@@ -53,6 +53,8 @@ def load() -> ctypes.CDLL:
     lib.attn_device_status.restype = i
     lib.attn_set_wait_timeout_ns.argtypes = [u64]
     lib.attn_set_wait_timeout_ns.restype = u64
+    lib.attn_selftest_exp2.argtypes = [vp, vp, i, vp]
+    lib.attn_selftest_exp2.restype = i
     lib.attn_selftest_wait_timeout.argtypes = [u64, vp]
     lib.attn_selftest_wait_timeout.restype = i
     lib.attn_status_string.argtypes = [i]
@@ -168,3 +170,13 @@ def set_wait_timeout_ns(ns: int) -> int:
 
 def selftest_wait_timeout(ns: int, stream=None) -> int:
     return int(load().attn_selftest_wait_timeout(int(ns), _stream_ptr(stream)))
+
+
+def selftest_exp2(x: torch.Tensor) -> torch.Tensor:
+    """The fused pass's FMA-pipe 2^x, evaluated on a CUDA fp32 tensor."""
+    _check_dev(x, "x", torch.float32)
+    y = torch.empty_like(x)
+    st = load().attn_selftest_exp2(x.data_ptr(), y.data_ptr(), x.numel(), _stream_ptr(None))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_selftest_exp2")
+    return y

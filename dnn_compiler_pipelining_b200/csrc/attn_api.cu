@@ -284,6 +284,32 @@ __global__ void selftest_wait_kernel(uint64_t timeout_ns) {
 }
 }  // namespace attn_b200
 
+namespace attn_b200 {
+// The fast pass's FMA-pipe exponential, evaluated elementwise (pairs).
+__global__ void selftest_exp2_kernel(const float* x, float* y, int n) {
+  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (i + 1 < n) {
+    const float2 r = exp2_poly2(make_float2(x[i], x[i + 1]));
+    y[i] = r.x;
+    y[i + 1] = r.y;
+  } else if (i < n) {
+    y[i] = exp2_poly2(make_float2(x[i], x[i])).x;
+  }
+}
+}  // namespace attn_b200
+
+extern "C" attn_status attn_selftest_exp2(const float* x, float* y, int n, void* stream) {
+  if (!x || !y) return ATTN_ERR_NULL;
+  if (n < 0) return ATTN_ERR_SHAPE;
+  if (n == 0) return ATTN_OK;
+  int dev = 0;
+  attn_status st = device_setup(&dev);
+  if (st != ATTN_OK) return st;
+  const int pairs = (n + 1) / 2;
+  selftest_exp2_kernel<<<(pairs + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
 extern "C" attn_status attn_selftest_wait_timeout(uint64_t timeout_ns, void* stream) {
   int dev = 0;
   attn_status st = device_setup(&dev);

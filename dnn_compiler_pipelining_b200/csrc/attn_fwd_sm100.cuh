@@ -63,6 +63,11 @@ constexpr int kThreads = 512;
 constexpr uint32_t kTileBytes = kBlockM * kHeadDim * 2;  // 32 KiB fp16 tile
 constexpr uint32_t kPanelBytes = kTileBytes / 2;         // one 64-column swizzle panel
 constexpr float kRescaleLog2 = 8.0f;
+// Of every 8 column pairs, how many take 2^x from the FMA-pipe polynomial
+// instead of the MUFU unit.  Measured on B200 (B=64, S=8192 causal): 0, 2,
+// 3, 4 pairs gave 1000, 933, 899, 861 TFLOP/s, so the MUFU unit is not this
+// kernel's limit and the polynomial stays off.
+constexpr int kEmuPairs = 0;
 constexpr float kRedoThreshold = 3.98f;
 constexpr float kLn2 = 0.69314718055994531f;
 
@@ -522,14 +527,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int c = 0; c < 128; ++c)
               if (c > r) u[c] = 0xff800000u;  // -inf
           }
+          // row max: 8 independent chains of 3-input max, then a tree
           float mx8[8];
 #pragma unroll
           for (int t = 0; t < 8; ++t) mx8[t] = __uint_as_float(u[t]);
 #pragma unroll
-          for (int c = 8; c < 128; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(u[c]));
+          for (int c = 8; c < 128; c += 16)
 #pragma unroll
-          for (int t = 0; t < 4; ++t) mx8[t] = fmaxf(mx8[t], mx8[t + 4]);
-          const float cand = fmaxf(fmaxf(mx8[0], mx8[2]), fmaxf(mx8[1], mx8[3])) * sc;
+            for (int t = 0; t < 8; ++t)
+              mx8[t] = fmax3(mx8[t], __uint_as_float(u[c + t]), __uint_as_float(u[c + 8 + t]));
+          const float cand = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
+                                   fmaxf(mx8[6], mx8[7])) * sc;
           if (j == 0) {
             m_use = cand;
           } else {
@@ -555,15 +563,27 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float neg_m = -m_use;
           float lp[4] = {0.f, 0.f, 0.f, 0.f};
           if (!hilo) {
-            // P rounded to fp16; l sums exactly the rounded values
+            // P rounded to fp16; l sums exactly the rounded values.  In every
+            // 16 columns, kEmuPairs pairs take 2^x from the FMA-pipe
+            // polynomial and the rest from the MUFU unit.
+            const float2 sc2 = make_float2(sc, sc);
+            const float2 nm2 = make_float2(neg_m, neg_m);
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
               uint32_t ph[8];
 #pragma unroll
               for (int i = 0; i < 8; ++i) {
-                const float p0 = ex2_approx(fmaf(__uint_as_float(u[c * 16 + 2 * i]), sc, neg_m));
-                const float p1 = ex2_approx(fmaf(__uint_as_float(u[c * 16 + 2 * i + 1]), sc, neg_m));
-                ph[i] = pack_half2(p0, p1);
+                const float2 s2 = make_float2(__uint_as_float(u[c * 16 + 2 * i]),
+                                              __uint_as_float(u[c * 16 + 2 * i + 1]));
+                const float2 x2 = __ffma2_rn(s2, sc2, nm2);
+                float2 p2;
+                if (i < kEmuPairs) {
+                  p2 = exp2_poly2(x2);
+                } else {
+                  p2.x = ex2_approx(x2.x);
+                  p2.y = ex2_approx(x2.y);
+                }
+                ph[i] = pack_half2(p2.x, p2.y);
                 lp[i & 3] = add_half2_f32(ph[i], lp[i & 3]);
               }
               tmem_st8(s_t + c * 8, ph);

@@ -368,3 +368,38 @@ __device__ __forceinline__ void mma_f16_ts_off(uint32_t d_tmem, uint32_t a_tmem,
       : "memory");
 }
 }  // namespace attn_b200
+
+namespace attn_b200 {
+// max(a, b, c) in one instruction.
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// 2^x for two values on the FMA pipe (relief for the MUFU unit).  Range
+// reduction: n = round(x) by adding 1.5 * 2^23 (the rounded integer lands in
+// the low mantissa bits of t), f = x - n in [-1/2, 1/2]; 2^f from a degree-3
+// polynomial fitted here by minimax on relative error (Lawson-weighted least
+// squares; max relative error 7.6e-5 in fp32 Horner form); 2^n is added to
+// the exponent field as the integer (t_bits << 23), whose high part is zero
+// because the constant's low 9 bits are zero.  Relative error <= 8e-5 for x in
+// [-125, 8]; x is first clamped to -126, so below -125 results are
+// non-negative and under 2^-124 (they round to 0 in fp16).  Callers keep
+// x <= 8.
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+  constexpr float c0 = 0.9999275803565979f, c1 = 0.6932516098022461f;
+  constexpr float c2 = 0.24261526763439178f, c3 = 0.05522262305021286f;
+  x.x = fmaxf(x.x, -126.0f);
+  x.y = fmaxf(x.y, -126.0f);
+  const float2 t = __fadd2_rn(x, make_float2(kRound, kRound));
+  const float2 n = __fadd2_rn(t, make_float2(-kRound, -kRound));
+  const float2 f = __ffma2_rn(n, make_float2(-1.0f, -1.0f), x);
+  float2 p = __ffma2_rn(make_float2(c3, c3), f, make_float2(c2, c2));
+  p = __ffma2_rn(p, f, make_float2(c1, c1));
+  p = __ffma2_rn(p, f, make_float2(c0, c0));
+  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
+                     __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
+}
+}  // namespace attn_b200

@@ -155,6 +155,15 @@ attn_status attn_selftest_wait_timeout(uint64_t timeout_ns, void* stream);
 attn_status attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, float* lse,
                              int B, int Hq, int Hkv, int S, int D, int causal, void* stream);
 
+/*
+ * attn_selftest_exp2 -- evaluates, on the device, the polynomial 2^x that
+ * the fused pass uses for part of its exponentials (so tests can check it
+ * against a reference exp2).  x, y: device fp32 arrays of n elements
+ * (y = 2^x for x <= 8; x below -126 gives a non-negative value below 2^-125).
+ * Asynchronous on `stream`.
+ */
+attn_status attn_selftest_exp2(const float* x, float* y, int n, void* stream);
+
 /* Human-readable name of a status code (static storage, never NULL). */
 const char* attn_status_string(attn_status status);
 

@@ -173,3 +173,22 @@ def test_large_outputs_overflow_scan():
     parity.sampled_check(q, k, v, o, lse, True, n_random=512, seed=25, full_heads=True)
     # the list is empty again: a plain call right after still passes
     parity.full_check(1, 2, 1, 256, 128, True, seed=26)
+
+
+def test_fma_pipe_exp2_error_bound():
+    """The polynomial 2^x available to the fused pass for part of its
+    exponentials: relative error <= 8e-5 against fp64 exp2 for x in
+    [-125, 8] (results of normal fp32 range), and non-negative results below
+    2^-124 (they round to 0 in fp16) further down, including -inf."""
+    g = torch.Generator(device="cuda")
+    g.manual_seed(5)
+    x = torch.cat([torch.linspace(-125.0, 8.0, 1 << 20, device="cuda"),
+                   torch.rand(1 << 20, generator=g, device="cuda") * 133.0 - 125.0,
+                   torch.arange(-125, 9, device="cuda", dtype=torch.float32)])
+    y = attn.selftest_exp2(x)
+    ref = torch.exp2(x.double())
+    rel = ((y.double() - ref) / ref).abs().max().item()
+    assert rel <= 8e-5, rel
+    lo = attn.selftest_exp2(torch.tensor([-125.3, -125.9, -126.0, -127.0, -200.0, -1e30,
+                                          float("-inf")], device="cuda"))
+    assert torch.all(lo >= 0) and torch.all(lo < 2.0 ** -124), lo
