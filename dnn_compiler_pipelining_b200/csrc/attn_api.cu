@@ -95,7 +95,9 @@ attn_status device_setup(int* dev_out) {
     if (cudaDeviceGetAttribute(&g_dev_sms[dev], cudaDevAttrMultiProcessorCount, dev) !=
         cudaSuccess)
       return ATTN_ERR_CUDA;
-    if (cudaFuncSetAttribute(attn_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(attn_fwd_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(fwd_smem_bytes())) != cudaSuccess ||
+        cudaFuncSetAttribute(attn_fwd_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(fwd_smem_bytes())) != cudaSuccess)
       return ATTN_ERR_CUDA;
     g_dev_state[dev].store(1, std::memory_order_release);
@@ -204,12 +206,10 @@ attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float
 
   // fast pass over every item, then the hi+lo pass over the items it listed
   const int sms = g_dev_sms[dev];
-  p.mode = 0;
-  attn_fwd_kernel<<<p.n_items < sms ? p.n_items : sms, kThreads, fwd_smem_bytes(), cs>>>(tm_q, tm_k,
-                                                                                       tm_v, p);
+  attn_fwd_kernel<0><<<p.n_items < sms ? p.n_items : sms, kThreads, fwd_smem_bytes(), cs>>>(
+      tm_q, tm_k, tm_v, p);
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
-  p.mode = 1;
-  attn_fwd_kernel<<<sms, kThreads, fwd_smem_bytes(), cs>>>(tm_q, tm_k, tm_v, p);
+  attn_fwd_kernel<1><<<sms, kThreads, fwd_smem_bytes(), cs>>>(tm_q, tm_k, tm_v, p);
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
   return ATTN_OK;
 }
@@ -396,12 +396,10 @@ extern "C" attn_status attn_fwd_noalloc(const void* q, const void* k, const void
   if (cudaMemsetAsync(scratch, 0, kRedoHeaderWords * sizeof(unsigned int), cs) != cudaSuccess)
     return ATTN_ERR_CUDA;
   const int sms = g_dev_sms[dev];
-  p.mode = 0;
-  attn_fwd_kernel<<<p.n_items < sms ? p.n_items : sms, kThreads, fwd_smem_bytes(), cs>>>(tm_q, tm_k,
-                                                                                       tm_v, p);
+  attn_fwd_kernel<0><<<p.n_items < sms ? p.n_items : sms, kThreads, fwd_smem_bytes(), cs>>>(
+      tm_q, tm_k, tm_v, p);
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
-  p.mode = 1;
-  attn_fwd_kernel<<<sms, kThreads, fwd_smem_bytes(), cs>>>(tm_q, tm_k, tm_v, p);
+  attn_fwd_kernel<1><<<sms, kThreads, fwd_smem_bytes(), cs>>>(tm_q, tm_k, tm_v, p);
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
   return ATTN_OK;
 }

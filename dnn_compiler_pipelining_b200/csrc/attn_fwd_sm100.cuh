@@ -93,7 +93,6 @@ struct FwdParams {
   float* lse;
   int B, Hq, Hkv, S;
   int causal;
-  int mode;          // 0: fast pass; 1: redo listed items with hi+lo P
   int n_items;       // B * Hq * n_qb2
   int n_qb;          // S / 128 row blocks
   int n_qb2;         // ceil(n_qb / 2) items per (batch, head)
@@ -166,9 +165,10 @@ __device__ __forceinline__ Item decode_item(const FwdParams& p, int id) {
 }
 
 // k-th work item of this CTA, or -1 when done.
+template <int kMode>
 __device__ __forceinline__ int work_item(const FwdParams& p, int k, unsigned int n_listed) {
   const long long idx = static_cast<long long>(blockIdx.x) + static_cast<long long>(k) * gridDim.x;
-  if (p.mode == 1 && n_listed <= p.redo_capacity) {
+  if (kMode == 1 && n_listed <= p.redo_capacity) {
     if (idx >= n_listed) return -1;
     const unsigned int id = p.redo[kRedoHeaderWords + idx];
     // an id from another call's list (left by a launch that failed) is
@@ -237,6 +237,9 @@ __device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint3
   pv_step<7>(o_tmem, p_tmem, vd, idesc, acc);
 }
 
+// kMode 0: the fused pass over every item; kMode 1: the redo pass over the
+// listed items with hi + lo probabilities.
+template <int kMode>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
@@ -248,7 +251,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint64_t to = p.timeout_ns;
 
   if (threadIdx.x == 0) {
-    sm->n_listed = (p.mode == 1) ? *reinterpret_cast<volatile unsigned int*>(p.redo) : 0u;
+    sm->n_listed = (kMode == 1) ? *reinterpret_cast<volatile unsigned int*>(p.redo) : 0u;
     mbar_init(smem_addr(&sm->q_full), 1);
     mbar_init(smem_addr(&sm->q_empty), 1);
     for (int s = 0; s < kStages; ++s) {
@@ -272,7 +275,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   __syncthreads();
   const unsigned int n_listed = sm->n_listed;
-  const bool has_work = work_item(p, 0, n_listed) >= 0;
+  const bool has_work = work_item<kMode>(p, 0, n_listed) >= 0;
 
   if (has_work) {
     if (warp == kMmaWarp) {
@@ -302,7 +305,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         int k = 0;
         int item;
         bool ok = true;
-        for (; ok && (item = work_item(p, k, n_listed)) >= 0; ++k) {
+        for (; ok && (item = work_item<kMode>(p, k, n_listed)) >= 0; ++k) {
           const Item it = decode_item(p, item);
           if (!is_v) {
             if (k > 0 &&
@@ -347,13 +350,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       } else if (warp == kMmaWarp && lane == 0) {
         // ------------------------------------------------------------ MMA issuer
-        const bool hilo = p.mode == 1;
+        constexpr bool hilo = kMode == 1;
         int rc = 0;
         int pcnt[2] = {0, 0};
         int acnt[2] = {0, 0};  // items so far in which tile X was active
         bool ok = true;
         int item;
-        for (int k = 0; ok && (item = work_item(p, k, n_listed)) >= 0; ++k) {
+        for (int k = 0; ok && (item = work_item<kMode>(p, k, n_listed)) >= 0; ++k) {
           const Item it = decode_item(p, item);
           const int n_b = it.n_blocks;
           if (!mbar_wait(smem_addr(&sm->q_full), k & 1, abort, to, kSiteMmaQ)) {
@@ -419,7 +422,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
       int acnt[2] = {0, 0};  // items so far in which tile X was active
       int item;
-      for (int k = 0; (item = work_item(p, k, n_listed)) >= 0; ++k) {
+      for (int k = 0; (item = work_item<kMode>(p, k, n_listed)) >= 0; ++k) {
         const Item it = decode_item(p, item);
         bool flag = false;
         bool ok = true;
@@ -467,7 +470,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           flag |= omax >= kRedoThreshold;
         }
         if (!ok) break;
-        if (p.mode == 0) {
+        if (kMode == 0) {
           // One redo-list entry per item if any of its rows needs it.  The
           // last of the four epilogue warps to finish the item appends it (no
           // barrier, so a warp that gave up on a wait cannot block the
@@ -497,11 +500,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t s_t = lane_base + tmem_s_col(x);
       const uint32_t o_t = lane_base + tmem_o_col(x);
       const float sc = p.scale_log2;
-      const bool hilo = p.mode == 1;
+      constexpr bool hilo = kMode == 1;
       int scnt = 0;
       int acnt = 0;  // items so far in which this tile was active
       int item;
-      for (int k = 0; (item = work_item(p, k, n_listed)) >= 0; ++k) {
+      for (int k = 0; (item = work_item<kMode>(p, k, n_listed)) >= 0; ++k) {
         const Item it = decode_item(p, item);
         const int n_x = it.n_kv[x];
         if (n_x == 0) continue;
@@ -562,7 +565,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           const float neg_m = -m_use;
           float lp[4] = {0.f, 0.f, 0.f, 0.f};
-          if (!hilo) {
+          if constexpr (!hilo) {
             // P rounded to fp16; l sums exactly the rounded values.  In every
             // 16 columns, kEmuPairs pairs take 2^x from the FMA-pipe
             // polynomial and the rest from the MUFU unit.
@@ -627,7 +630,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
-  if (p.mode == 1) {
+  if (kMode == 1) {
     // the last CTA out empties the redo list for the next call on this stream
     __syncthreads();
     if (threadIdx.x == 0) {
