@@ -69,9 +69,7 @@ unsigned int* redo_list(int dev, cudaStream_t stream) {
   return static_cast<unsigned int*>(ptr);
 }
 
-size_t fwd_smem_bytes() {
-  return sizeof(SharedFwd) + 1024;  // + slack to align the base to 1 KiB
-}
+size_t fwd_smem_bytes() { return sizeof(SharedFwd); }  // the kernel checks 1 KiB alignment
 
 attn_status device_setup(int* dev_out) {
   int dev = 0;
@@ -232,6 +230,7 @@ attn_status attn_device_status(void* stream, uint32_t* site) {
     if (cudaMemcpyToSymbol(g_attn_status, zero, sizeof(zero)) != cudaSuccess) return ATTN_ERR_CUDA;
   }
   if (site) *site = words[1];
+  if (words[0] & kStatusSmemAlign) return ATTN_ERR_CUDA;
   return (words[0] & kStatusTimeout) ? ATTN_ERR_DEVICE_TIMEOUT : ATTN_OK;
 }
 

@@ -58,7 +58,8 @@ constexpr int kBlockM = 128;   // query rows per tile
 constexpr int kBlockN = 128;   // keys per K/V tile
 constexpr int kHeadDim = 128;  // D
 constexpr int kItemRows = 2 * kBlockM;
-constexpr int kStages = 2;     // K/V ring depth
+constexpr int kStagesK = 3;    // K ring depth
+constexpr int kStagesV = 2;    // V ring depth (V_j is needed one softmax later than K_j)
 constexpr int kThreads = 512;
 constexpr uint32_t kTileBytes = kBlockM * kHeadDim * 2;  // 32 KiB fp16 tile
 constexpr uint32_t kPanelBytes = kTileBytes / 2;         // one 64-column swizzle panel
@@ -113,20 +114,24 @@ enum WaitSite : uint32_t {
   kSiteMmaP = 0x204,
   kSiteMmaO = 0x205,
   kSiteSoftmaxS = 0x301,
+  kSiteSoftmaxStats = 0x302,
   kSiteEpilogueO = 0x401,
   kSiteEpilogueStats = 0x402,
   kSiteDrain = 0x501,
 };
 
-struct alignas(1024) SharedFwd {
+// Shared memory: 224 KiB of tiles first (each 1 KiB aligned, as the 128-byte
+// swizzle needs), then the row statistics and the barriers.  The dynamic
+// shared memory base is checked to be 1 KiB aligned at launch.
+struct SharedFwd {
   uint8_t q[2][kTileBytes];
-  uint8_t k[kStages][kTileBytes];
-  uint8_t v[kStages][kTileBytes];
-  float stat_m[2][2][kBlockM];  // [parity of the tile's active-item count][tile][row]
-  float stat_l[2][2][kBlockM];
+  uint8_t k[kStagesK][kTileBytes];
+  uint8_t v[kStagesV][kTileBytes];
+  float stat_m[2][kBlockM];  // [tile][row], handed from softmax to epilogue
+  float stat_l[2][kBlockM];
   uint64_t q_full, q_empty;
-  uint64_t k_full[kStages], v_full[kStages], k_empty[kStages], v_empty[kStages];
-  uint64_t s_full[2], p_full[2], o_done[2], o_free[2], stats_ready[2];
+  uint64_t k_full[kStagesK], k_empty[kStagesK], v_full[kStagesV], v_empty[kStagesV];
+  uint64_t s_full[2], p_full[2], o_done[2], o_free[2], stats_ready[2], stats_free[2];
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
@@ -134,6 +139,8 @@ struct alignas(1024) SharedFwd {
   int item_warps[2];  // [item parity]: epilogue warps done with the item
   unsigned int n_listed;
 };
+
+static_assert(sizeof(SharedFwd) <= 232448, "shared memory exceeds the 227 KiB per-block limit");
 
 struct Item {
   int b, hq, g, qb2;
@@ -183,7 +190,10 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64
   mbar_wait(bar, parity, &never, timeout_ns, kSiteDrain);
 }
 
-__device__ __forceinline__ uint32_t ring_parity(int rc) { return (rc / kStages) & 1; }
+template <int kDepth>
+__device__ __forceinline__ uint32_t ring_parity(int rc) {
+  return (rc / kDepth) & 1;
+}
 
 // S_X(j) = Q_X K^T: 8 MMAs of K = 16 over the head dimension.  Both operands
 // are K-major; 16 columns are 32 bytes inside a 128-byte swizzled row and
@@ -243,21 +253,27 @@ template <int kMode>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
-  extern __shared__ uint8_t smem_raw[];
-  SharedFwd* sm = reinterpret_cast<SharedFwd*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                               ~static_cast<uintptr_t>(1023));
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  SharedFwd* sm = reinterpret_cast<SharedFwd*>(smem_raw);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const uint64_t to = p.timeout_ns;
+  if (smem_addr(smem_raw) & 1023u) {
+    // the swizzled tiles need a 1 KiB aligned base; report instead of computing garbage
+    if (threadIdx.x == 0) atomicOr(&g_attn_status[0], kStatusSmemAlign);
+    return;
+  }
 
   if (threadIdx.x == 0) {
     sm->n_listed = (kMode == 1) ? *reinterpret_cast<volatile unsigned int*>(p.redo) : 0u;
     mbar_init(smem_addr(&sm->q_full), 1);
     mbar_init(smem_addr(&sm->q_empty), 1);
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < kStagesK; ++s) {
       mbar_init(smem_addr(&sm->k_full[s]), 1);
-      mbar_init(smem_addr(&sm->v_full[s]), 1);
       mbar_init(smem_addr(&sm->k_empty[s]), 1);
+    }
+    for (int s = 0; s < kStagesV; ++s) {
+      mbar_init(smem_addr(&sm->v_full[s]), 1);
       mbar_init(smem_addr(&sm->v_empty[s]), 1);
     }
     for (int x = 0; x < 2; ++x) {
@@ -266,6 +282,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(smem_addr(&sm->o_done[x]), 1);
       mbar_init(smem_addr(&sm->o_free[x]), kBlockM);
       mbar_init(smem_addr(&sm->stats_ready[x]), kBlockM);
+      mbar_init(smem_addr(&sm->stats_free[x]), kBlockM);
     }
     mbar_init(smem_addr(&sm->drain), 1);
     sm->abort = 0;
@@ -325,10 +342,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           const int kv_row = (it.b * p.Hkv + it.g) * p.S;
           for (int j = 0; j < it.n_blocks; ++j, ++rc) {
-            const int st = rc % kStages;
+            const int depth = is_v ? kStagesV : kStagesK;
+            const int st = rc % depth;
             const uint32_t empty = smem_addr(is_v ? &sm->v_empty[st] : &sm->k_empty[st]);
-            if (rc >= kStages && !mbar_wait(empty, ring_parity(rc) ^ 1, abort, to,
-                                            is_v ? kSiteProducerV : kSiteProducerK)) {
+            if (rc >= depth && !mbar_wait(empty, ((rc / depth) & 1) ^ 1, abort, to,
+                                          is_v ? kSiteProducerV : kSiteProducerK)) {
               ok = false;
               break;
             }
@@ -344,9 +362,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           // every copy still in flight must land before the CTA exits: the
           // last Q load and the last load of each ring stage
           if (!is_v && k > 0) drain_wait(smem_addr(&sm->q_full), (k - 1) & 1, to);
-          for (int t = (rc > kStages ? rc - kStages : 0); t < rc; ++t)
-            drain_wait(smem_addr(is_v ? &sm->v_full[t % kStages] : &sm->k_full[t % kStages]),
-                       ring_parity(t), to);
+          const int depth = is_v ? kStagesV : kStagesK;
+          for (int t = (rc > depth ? rc - depth : 0); t < rc; ++t)
+            drain_wait(smem_addr(is_v ? &sm->v_full[t % depth] : &sm->k_full[t % depth]),
+                       ((t / depth) & 1), to);
         }
       } else if (warp == kMmaWarp && lane == 0) {
         // ------------------------------------------------------------ MMA issuer
@@ -364,32 +383,25 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           for (int j = 0; ok && j <= n_b; ++j) {
-            const int st_k = (rc + j) % kStages;
-            const int st_v = (rc + j + kStages - 1) % kStages;
-            if (j < n_b &&
-                !mbar_wait(smem_addr(&sm->k_full[st_k]), ring_parity(rc + j), abort, to, kSiteMmaK)) {
-              ok = false;
-              break;
-            }
-            if (j >= 1 && !mbar_wait(smem_addr(&sm->v_full[st_v]), ring_parity(rc + j - 1), abort,
-                                     to, kSiteMmaV)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
+            // step j: PV_X(j-1) then S_X(j) for each tile; V_{j-1} and K_j are
+            // awaited just before the first MMA that reads them
+            const int st_k = (rc + j) % kStagesK;
+            const int st_v = (rc + j + kStagesV - 1) % kStagesV;
+            bool have_k = false, have_v = false;
             for (int x = 0; ok && x < 2; ++x) {
               const int n_x = it.n_kv[x];
               if (j >= 1 && j - 1 < n_x) {
+                if (!have_v) {
+                  ok = mbar_wait(smem_addr(&sm->v_full[st_v]), ring_parity<kStagesV>(rc + j - 1),
+                                 abort, to, kSiteMmaV);
+                  have_v = true;
+                }
                 // the epilogue must have read O_X of the tile's previous item
-                if (j == 1 && acnt[x] > 0 &&
-                    !mbar_wait(smem_addr(&sm->o_free[x]), (acnt[x] - 1) & 1, abort, to, kSiteMmaO)) {
-                  ok = false;
-                  break;
-                }
-                if (!mbar_wait(smem_addr(&sm->p_full[x]), pcnt[x] & 1, abort, to, kSiteMmaP)) {
-                  ok = false;
-                  break;
-                }
+                ok = ok && (j != 1 || acnt[x] == 0 ||
+                            mbar_wait(smem_addr(&sm->o_free[x]), (acnt[x] - 1) & 1, abort, to,
+                                      kSiteMmaO));
+                ok = ok && mbar_wait(smem_addr(&sm->p_full[x]), pcnt[x] & 1, abort, to, kSiteMmaP);
+                if (!ok) break;
                 ++pcnt[x];
                 tc_fence_after();
                 const uint32_t v_s = smem_addr(sm->v[st_v]);
@@ -398,6 +410,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (j == n_x) tc_commit(smem_addr(&sm->o_done[x]));
               }
               if (j < n_x) {
+                if (!have_k) {
+                  ok = mbar_wait(smem_addr(&sm->k_full[st_k]), ring_parity<kStagesK>(rc + j), abort,
+                                 to, kSiteMmaK);
+                  have_k = true;
+                  if (!ok) break;
+                  tc_fence_after();
+                }
                 issue_qk(tmem + tmem_s_col(x), smem_addr(sm->q[x]), smem_addr(sm->k[st_k]));
                 tc_commit(smem_addr(&sm->s_full[x]));
               }
@@ -437,8 +456,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           tc_fence_after();
-          const float m_use = sm->stat_m[a & 1][x][r];
-          const float l = sm->stat_l[a & 1][x][r];
+          const float m_use = sm->stat_m[x][r];
+          const float l = sm->stat_l[x][r];
+          mbar_arrive(smem_addr(&sm->stats_free[x]));  // the softmax may write the next item's
           const float inv_l = 1.0f / l;
           const int row = (it.b * p.Hq + it.hq) * p.S + it.qb2 * kItemRows + x * kBlockM + r;
           uint4* orow = reinterpret_cast<uint4*>(p.o + static_cast<size_t>(row) * kHeadDim);
@@ -615,8 +635,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive(smem_addr(&sm->p_full[x]));
         }
         if (!ok) break;
-        sm->stat_m[acnt & 1][x][r] = m_use;
-        sm->stat_l[acnt & 1][x][r] = l;
+        // the epilogue must have read this tile's previous statistics
+        ok = acnt == 0 ||
+             mbar_wait(smem_addr(&sm->stats_free[x]), (acnt - 1) & 1, abort, to, kSiteSoftmaxStats);
+        if (!__all_sync(0xffffffffu, ok)) break;
+        sm->stat_m[x][r] = m_use;
+        sm->stat_l[x][r] = l;
         ++acnt;
         mbar_arrive(smem_addr(&sm->stats_ready[x]));
       }

@@ -66,6 +66,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // this definition; the host reads it with cudaMemcpyFromSymbol.
 __device__ unsigned int g_attn_status[2];
 constexpr unsigned int kStatusTimeout = 1u;
+constexpr unsigned int kStatusSmemAlign = 2u;  // dynamic shared memory base not 1 KiB aligned
 
 // Waits until phase `parity` of the barrier has completed.  Bounded: after
 // `timeout_ns` of wall time, or as soon as another role of the CTA has given
