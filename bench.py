@@ -379,7 +379,7 @@ def run_gpu(args, w, name):
             "scaling": "weak", "vs_baseline": None, "dtype": "f16",
             "data": "synthetic", "config": workload_config(w, name, world),
             "e2e": e2e, "roofline": roofline, "cpu_baseline": cpu, "clocks": clocks,
-            "gpu_launches": args.steps,
+            "gpu_launches": 2 * args.steps,  # per step: the fused pass and the redo pass
             "pct_of_nominal_fp16_peak": 100.0 * value / world / NOMINAL_DENSE_FP16_TFLOPS,
         }
         print(json.dumps(line), flush=True)
