@@ -14,6 +14,7 @@
 #include <utility>
 
 #include "attn.h"
+#include "attn_fwd_pair_sm100.cuh"
 #include "attn_fwd_sm100.cuh"
 
 namespace attn_b200 {
@@ -41,6 +42,7 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 // memory opt-in.  0 = not done, 1 = ok, 2 = unsupported device.
 std::atomic<int> g_dev_state[kMaxDevices];
 int g_dev_sms[kMaxDevices];
+int g_dev_pairs[kMaxDevices];  // 2-CTA clusters of the pair kernel resident at once
 std::mutex g_dev_mutex;
 
 // Redo lists (items the fast pass hands to the hi+lo pass), one per
@@ -70,6 +72,7 @@ unsigned int* redo_list(int dev, cudaStream_t stream) {
 }
 
 size_t fwd_smem_bytes() { return sizeof(SharedFwd); }  // the kernel checks 1 KiB alignment
+size_t pair_smem_bytes() { return sizeof(pair::SharedPair); }
 
 attn_status device_setup(int* dev_out) {
   int dev = 0;
@@ -96,8 +99,20 @@ attn_status device_setup(int* dev_out) {
     if (cudaFuncSetAttribute(attn_fwd_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(fwd_smem_bytes())) != cudaSuccess ||
         cudaFuncSetAttribute(attn_fwd_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(fwd_smem_bytes())) != cudaSuccess)
+                             static_cast<int>(fwd_smem_bytes())) != cudaSuccess ||
+        cudaFuncSetAttribute(pair::attn_fwd_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(pair_smem_bytes())) != cudaSuccess)
       return ATTN_ERR_CUDA;
+    // a persistent grid of as many CTA pairs as can be resident together
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * (g_dev_sms[dev] / 2));
+    cfg.blockDim = dim3(pair::kThreads);
+    cfg.dynamicSmemBytes = pair_smem_bytes();
+    int pairs = 0;
+    if (cudaOccupancyMaxActiveClusters(&pairs, pair::attn_fwd_pair_kernel, &cfg) != cudaSuccess ||
+        pairs < 1)
+      return ATTN_ERR_CUDA;
+    g_dev_pairs[dev] = pairs;
     g_dev_state[dev].store(1, std::memory_order_release);
   }
   return g_dev_state[dev].load() == 1 ? ATTN_OK : ATTN_ERR_UNSUPPORTED;
@@ -105,12 +120,13 @@ attn_status device_setup(int* dev_out) {
 
 // 2-D view [rows, 128] fp16 of a dense [.., S, 128] tensor; 64 x 128 boxes
 // (one 128-byte swizzle panel of 128 rows).
-bool encode_rows_map(CUtensorMap* map, const void* base, uint64_t rows) {
+bool encode_rows_map(CUtensorMap* map, const void* base, uint64_t rows,
+                     uint32_t box_rows = kBlockM) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(kHeadDim), static_cast<cuuint64_t>(rows)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(kHeadDim) * 2};
-  cuuint32_t box[2] = {64, static_cast<cuuint32_t>(kBlockM)};
+  cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides,
                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -133,6 +149,43 @@ attn_status validate_sizes(int B, int Hq, int Hkv, int S, int D) {
 }
 
 size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+// Tensor maps of one call: Q and V in 128-row boxes, K in 64-row boxes (the
+// pair pass loads half a key block per CTA) and 128-row boxes (redo pass).
+struct CallMaps {
+  CUtensorMap q, k, k_half, v;
+};
+
+bool encode_call_maps(CallMaps* m, const void* q, const void* k, const void* v, int B, int Hq,
+                      int Hkv, int S) {
+  const uint64_t q_rows = static_cast<uint64_t>(B) * Hq * S;
+  const uint64_t kv_rows = static_cast<uint64_t>(B) * Hkv * S;
+  return encode_rows_map(&m->q, q, q_rows) && encode_rows_map(&m->k, k, kv_rows) &&
+         encode_rows_map(&m->k_half, k, kv_rows, kBlockM / 2) && encode_rows_map(&m->v, v, kv_rows);
+}
+
+// Which kernel runs the fused pass: the single-CTA kernel (attn_fwd_kernel<0>)
+// or the CTA-pair kernel (pair::attn_fwd_pair_kernel), which computes the
+// same items.
+constexpr bool kPairFusedPass = false;
+
+// The fused pass over every item, then the hi+lo pass over the items it
+// listed.
+attn_status launch_passes(const CallMaps& m, const FwdParams& p, int dev, cudaStream_t cs) {
+  if (kPairFusedPass) {
+    const int pairs = p.n_items < g_dev_pairs[dev] ? p.n_items : g_dev_pairs[dev];
+    pair::attn_fwd_pair_kernel<<<2 * pairs, pair::kThreads, pair_smem_bytes(), cs>>>(
+        m.q, m.k_half, m.v, p);
+  } else {
+    const int sms = g_dev_sms[dev];
+    attn_fwd_kernel<0><<<p.n_items < sms ? p.n_items : sms, kThreads, fwd_smem_bytes(), cs>>>(
+        m.q, m.k, m.v, p);
+  }
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  attn_fwd_kernel<1><<<g_dev_sms[dev], kThreads, fwd_smem_bytes(), cs>>>(m.q, m.k, m.v, p);
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  return ATTN_OK;
+}
 
 }  // namespace
 }  // namespace attn_b200
@@ -177,11 +230,8 @@ attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float
   st = device_setup(&dev);
   if (st != ATTN_OK) return st;
 
-  CUtensorMap tm_q, tm_k, tm_v;
-  if (!encode_rows_map(&tm_q, q, static_cast<uint64_t>(B) * Hq * S) ||
-      !encode_rows_map(&tm_k, k, static_cast<uint64_t>(B) * Hkv * S) ||
-      !encode_rows_map(&tm_v, v, static_cast<uint64_t>(B) * Hkv * S))
-    return ATTN_ERR_CUDA;
+  CallMaps maps;
+  if (!encode_call_maps(&maps, q, k, v, B, Hq, Hkv, S)) return ATTN_ERR_CUDA;
 
   FwdParams p;
   p.o = static_cast<__half*>(o);
@@ -202,14 +252,7 @@ attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float
   if (!p.redo) return ATTN_ERR_CUDA;
   p.redo_capacity = kRedoCapacity;
 
-  // fast pass over every item, then the hi+lo pass over the items it listed
-  const int sms = g_dev_sms[dev];
-  attn_fwd_kernel<0><<<p.n_items < sms ? p.n_items : sms, kThreads, fwd_smem_bytes(), cs>>>(
-      tm_q, tm_k, tm_v, p);
-  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
-  attn_fwd_kernel<1><<<sms, kThreads, fwd_smem_bytes(), cs>>>(tm_q, tm_k, tm_v, p);
-  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
-  return ATTN_OK;
+  return launch_passes(maps, p, dev, cs);
 }
 
 size_t attn_fwd_host_workspace_bytes(int B, int Hq, int Hkv, int S, int D) {
@@ -367,11 +410,8 @@ extern "C" attn_status attn_fwd_noalloc(const void* q, const void* k, const void
   unsigned int* scratch = noalloc_scratch(dev);
   if (!scratch) return ATTN_ERR_CUDA;
 
-  CUtensorMap tm_q, tm_k, tm_v;
-  if (!encode_rows_map(&tm_q, q, static_cast<uint64_t>(B) * Hq * S) ||
-      !encode_rows_map(&tm_k, k, static_cast<uint64_t>(B) * Hkv * S) ||
-      !encode_rows_map(&tm_v, v, static_cast<uint64_t>(B) * Hkv * S))
-    return ATTN_ERR_CUDA;
+  CallMaps maps;
+  if (!encode_call_maps(&maps, q, k, v, B, Hq, Hkv, S)) return ATTN_ERR_CUDA;
 
   FwdParams p;
   p.o = static_cast<__half*>(o);
@@ -394,11 +434,5 @@ extern "C" attn_status attn_fwd_noalloc(const void* q, const void* k, const void
   // the shared array keeps the previous call's header: start from an empty list
   if (cudaMemsetAsync(scratch, 0, kRedoHeaderWords * sizeof(unsigned int), cs) != cudaSuccess)
     return ATTN_ERR_CUDA;
-  const int sms = g_dev_sms[dev];
-  attn_fwd_kernel<0><<<p.n_items < sms ? p.n_items : sms, kThreads, fwd_smem_bytes(), cs>>>(
-      tm_q, tm_k, tm_v, p);
-  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
-  attn_fwd_kernel<1><<<sms, kThreads, fwd_smem_bytes(), cs>>>(tm_q, tm_k, tm_v, p);
-  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
-  return ATTN_OK;
+  return launch_passes(maps, p, dev, cs);
 }

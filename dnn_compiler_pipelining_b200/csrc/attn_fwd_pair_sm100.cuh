@@ -1,0 +1,595 @@
+// attn_fwd_pair_sm100.cuh -- the fused attention forward pass on CTA pairs.
+//
+// Same computation as attn_fwd_sm100.cuh (O = softmax(Q K^T / sqrt(D)
+// [+ causal mask]) V and the row log-sum-exp; the FlashAttention forward that
+// the PipeThreader pages evaluate, papers.lqhl.me "PipeThreader-OSDI25",
+// section 实验与结果, paper Sec. 6.2 / Fig. 12), with its load / mma /
+// softmax tasks mapped onto two SMs at once:
+//
+// A 2-CTA cluster takes one work item, 256 query rows of one (batch, query
+// head); CTA r of the pair owns rows [128 r, 128 r + 128) of the item.  The
+// even CTA issues every MMA as tcgen05.mma.cta_group::2 with M = 256: each
+// CTA holds its own 128 rows of Q (and of S, P, O in its own TMEM) but only
+// half of each key block's operand -- 64 of the 128 keys of K_j, and 64 of
+// the 128 head-dimension columns of V_j -- so every K/V byte crosses from L2
+// into shared memory once per pair, not once per SM.
+//
+// Each CTA's TMEM (512 columns) holds two S buffers and two O buffers:
+//   S[0] [0,128)  S[1] [128,256)   (key block g of the pair's block
+//   sequence goes to S[g & 1]; P_g, fp16, is written over its first 64
+//   columns)
+//   O[0] [256,384) O[1] [384,512)  (item k accumulates in O[k & 1])
+// With S double-buffered the MMA warp issues S(g+1) before PV(g): the
+// softmax of block g+1 never waits for PV(g), and the tensor core computes
+// S(g+1) while the softmax works on block g.  With O double-buffered the
+// epilogue of item k overlaps item k+1.  Q is double-buffered too, so the
+// next item's Q is in shared memory before its first S.
+//
+// Warp roles (384 threads per CTA):
+//   warps 0-3   softmax (one query row per thread = TMEM lane)
+//   warps 4-7   epilogue: O / l -> fp16, LSE
+//   warp 8      TMA producer of Q (per item) and this CTA's half of K_j
+//   warp 9      MMA issuer (even CTA, one thread); TMEM allocation (both)
+//   warp 10     TMA producer of this CTA's half of V_j
+//   warp 11     idle
+//
+// Signals between the two CTAs: the odd CTA's loads complete their bytes
+// on the even CTA's "full" barriers; the even CTA's commits arrive on the
+// barrier of the same offset in both CTAs (multicast); the odd CTA's
+// softmax and epilogue warps arrive on the even CTA's p_full / o_free.
+#pragma once
+
+#include <cuda_fp16.h>
+
+#include "attn_fwd_sm100.cuh"
+#include "ptx_sm100.cuh"
+
+namespace attn_b200 {
+namespace pair {
+
+constexpr int kStagesK = 4;                            // K ring (this CTA's 64 keys of a block)
+constexpr int kStagesV = 4;                            // V ring (this CTA's 64 columns of a block)
+constexpr uint32_t kHalfBytes = kTileBytes / 2;        // 16 KiB
+constexpr uint32_t kKPanelBytes = kHalfBytes / 2;      // 64 keys x 64 columns
+constexpr int kThreads = 384;
+constexpr int kEpilogueWarp0 = 4;
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr int kProducerVWarp = 10;
+constexpr int kRegsSoftmax = 224;
+constexpr int kRegsEpilogue = 96;
+constexpr int kRegsOther = 56;
+static_assert(128 * kRegsSoftmax + 128 * kRegsEpilogue + 128 * kRegsOther <= 65536,
+              "register split exceeds the register file");
+constexpr uint16_t kBothCtas = 0x3;
+
+__device__ __forceinline__ uint32_t tmem_s(int b) { return static_cast<uint32_t>(b) * 128u; }
+__device__ __forceinline__ uint32_t tmem_o(int b) { return 256u + static_cast<uint32_t>(b) * 128u; }
+
+enum PairWaitSite : uint32_t {
+  kSitePairProducerQ = 0x1101,
+  kSitePairProducerK = 0x1102,
+  kSitePairProducerV = 0x1103,
+  kSitePairMmaQ = 0x1201,
+  kSitePairMmaK = 0x1202,
+  kSitePairMmaV = 0x1203,
+  kSitePairMmaP = 0x1204,
+  kSitePairMmaO = 0x1205,
+  kSitePairSoftmaxS = 0x1301,
+  kSitePairSoftmaxStats = 0x1302,
+  kSitePairSoftmaxPV = 0x1303,
+  kSitePairEpilogueO = 0x1401,
+  kSitePairEpilogueStats = 0x1402,
+  kSitePairDrain = 0x1501,
+};
+
+// Identical layout in both CTAs: the pair MMAs address the odd CTA's
+// operands and barriers at the even CTA's offsets.
+struct SharedPair {
+  uint8_t q[2][kTileBytes];         // [item parity] this CTA's 128 rows, two 64-column panels
+  uint8_t k[kStagesK][kHalfBytes];  // 64 keys x 128 columns, two panels of 8 KiB
+  uint8_t v[kStagesV][kHalfBytes];  // 128 keys x 64 columns (one panel)
+  float stat_m[2][kBlockM];         // [item parity][row]
+  float stat_l[2][kBlockM];
+  uint64_t q_full[2], q_empty[2];
+  uint64_t k_full[kStagesK], k_empty[kStagesK], v_full[kStagesV], v_empty[kStagesV];
+  uint64_t s_full[2], p_full[2], pv_done[2], o_done[2], o_free[2];
+  uint64_t stats_ready[2], stats_free[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+  int item_flag[2];
+  int item_warps[2];
+};
+static_assert(sizeof(SharedPair) <= 232448, "shared memory exceeds the 227 KiB per-block limit");
+
+// Work item of a pair: the same ids as the single-CTA pass (kv-head major,
+// 256-row blocks from last to first), so the redo list is shared.
+struct PairItem {
+  int b, hq, g, qb2;
+  bool half1;    // the odd CTA's 128 rows exist (S / 128 may be odd)
+  int n_blocks;  // key blocks the pair computes
+};
+
+__device__ __forceinline__ PairItem decode_pair_item(const FwdParams& p, int id) {
+  const int per_kv = p.group * p.n_qb2;
+  const int kvh = id / per_kv;
+  const int rem = id - kvh * per_kv;
+  PairItem it;
+  it.b = kvh / p.Hkv;
+  it.g = kvh - it.b * p.Hkv;
+  it.qb2 = p.n_qb2 - 1 - rem / p.group;
+  it.hq = it.g * p.group + rem % p.group;
+  it.half1 = 2 * it.qb2 + 1 < p.n_qb;
+  if (p.causal)
+    it.n_blocks = it.half1 ? 2 * it.qb2 + 2 : 2 * it.qb2 + 1;
+  else
+    it.n_blocks = p.n_qb;
+  return it;
+}
+
+// S(g) = Q K_j^T over the pair: 8 MMAs of K = 16.  Q panels are 16 KiB
+// apart, this CTA's K panels (64 rows) 8 KiB apart.
+template <int kk>
+__device__ __forceinline__ void qk_step_pair(uint32_t d_tmem, uint64_t qd, uint64_t kd,
+                                             uint32_t idesc) {
+  constexpr uint32_t a_off = ((kk >> 2) * kPanelBytes + (kk & 3) * 32) >> 4;
+  constexpr uint32_t b_off = ((kk >> 2) * kKPanelBytes + (kk & 3) * 32) >> 4;
+  mma_pair_ss_off<a_off, b_off>(d_tmem, qd, kd, idesc, kk > 0 ? 1u : 0u);
+}
+__device__ __forceinline__ void issue_qk_pair(uint32_t d_tmem, uint32_t q_s, uint32_t k_s) {
+  const uint32_t idesc = idesc_f16_f32(2 * kBlockM, kBlockN, false, false);
+  const uint64_t qd = smem_desc_sw128(q_s, 16, 1024);
+  const uint64_t kd = smem_desc_sw128(k_s, 16, 1024);
+  qk_step_pair<0>(d_tmem, qd, kd, idesc);
+  qk_step_pair<1>(d_tmem, qd, kd, idesc);
+  qk_step_pair<2>(d_tmem, qd, kd, idesc);
+  qk_step_pair<3>(d_tmem, qd, kd, idesc);
+  qk_step_pair<4>(d_tmem, qd, kd, idesc);
+  qk_step_pair<5>(d_tmem, qd, kd, idesc);
+  qk_step_pair<6>(d_tmem, qd, kd, idesc);
+  qk_step_pair<7>(d_tmem, qd, kd, idesc);
+}
+
+// O (+)= P V over the pair: A = P from each CTA's TMEM (8 columns = 16 keys
+// per MMA), B = V, MN-major; each CTA holds one 64-column panel of V_j.
+template <int kk>
+__device__ __forceinline__ void pv_step_pair(uint32_t o_tmem, uint32_t p_tmem, uint64_t vd,
+                                             uint32_t idesc, uint32_t acc) {
+  constexpr uint32_t a_off = kk * 8;
+  constexpr uint32_t b_off = (kk * 2048) / 16;
+  mma_pair_ts_off<a_off, b_off>(o_tmem, p_tmem, vd, idesc, (acc || kk > 0) ? 1u : 0u);
+}
+__device__ __forceinline__ void issue_pv_pair(uint32_t o_tmem, uint32_t p_tmem, uint32_t v_s,
+                                              bool accumulate) {
+  const uint32_t idesc = idesc_f16_f32(2 * kBlockM, kHeadDim, false, true);
+  const uint64_t vd = smem_desc_sw128(v_s, kPanelBytes, 1024);
+  const uint32_t acc = accumulate ? 1u : 0u;
+  pv_step_pair<0>(o_tmem, p_tmem, vd, idesc, acc);
+  pv_step_pair<1>(o_tmem, p_tmem, vd, idesc, acc);
+  pv_step_pair<2>(o_tmem, p_tmem, vd, idesc, acc);
+  pv_step_pair<3>(o_tmem, p_tmem, vd, idesc, acc);
+  pv_step_pair<4>(o_tmem, p_tmem, vd, idesc, acc);
+  pv_step_pair<5>(o_tmem, p_tmem, vd, idesc, acc);
+  pv_step_pair<6>(o_tmem, p_tmem, vd, idesc, acc);
+  pv_step_pair<7>(o_tmem, p_tmem, vd, idesc, acc);
+}
+
+__device__ __forceinline__ void pair_sleep_ns(uint64_t ns) {
+  const uint64_t t0 = global_timer_ns();
+  while (global_timer_ns() - t0 < ns) __nanosleep(1000);
+}
+
+// The fused pass on CTA pairs (records items for the redo pass exactly as
+// attn_fwd_kernel<0> does).  Launched with 2-CTA clusters; the grid is an
+// even number of CTAs, pair c taking items c, c + pairs, ...
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
+                         const __grid_constant__ CUtensorMap tm_k,
+                         const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  SharedPair* sm = reinterpret_cast<SharedPair*>(smem_raw);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint64_t to = p.timeout_ns;
+  // both CTAs of a pair take the same branch here (same kernel, same layout)
+  if (cluster_nctarank() != 2 || (smem_addr(smem_raw) & 1023u)) {
+    if (threadIdx.x == 0) atomicOr(&g_attn_status[0], kStatusSmemAlign);
+    return;
+  }
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair_id = blockIdx.x >> 1;
+  const int n_pairs = gridDim.x >> 1;
+
+  if (threadIdx.x == 0) {
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(smem_addr(&sm->q_full[b]), 1);
+      mbar_init(smem_addr(&sm->q_empty[b]), 1);
+      mbar_init(smem_addr(&sm->s_full[b]), 1);
+      mbar_init(smem_addr(&sm->p_full[b]), 8);   // 4 softmax warps x 2 CTAs
+      mbar_init(smem_addr(&sm->pv_done[b]), 1);
+      mbar_init(smem_addr(&sm->o_done[b]), 1);
+      mbar_init(smem_addr(&sm->o_free[b]), 8);   // 4 epilogue warps x 2 CTAs
+      mbar_init(smem_addr(&sm->stats_ready[b]), kBlockM);
+      mbar_init(smem_addr(&sm->stats_free[b]), kBlockM);
+    }
+    for (int s = 0; s < kStagesK; ++s) {
+      mbar_init(smem_addr(&sm->k_full[s]), 1);
+      mbar_init(smem_addr(&sm->k_empty[s]), 1);
+    }
+    for (int s = 0; s < kStagesV; ++s) {
+      mbar_init(smem_addr(&sm->v_full[s]), 1);
+      mbar_init(smem_addr(&sm->v_empty[s]), 1);
+    }
+    mbar_init(smem_addr(&sm->drain), 1);
+    sm->abort = 0;
+    sm->item_flag[0] = sm->item_flag[1] = 0;
+    sm->item_warps[0] = sm->item_warps[1] = 0;
+    fence_mbar_init();
+  }
+  // the other CTA's barriers exist before anything signals them
+  cluster_sync();
+  if (pair_id >= p.n_items) return;  // same for both CTAs of the pair
+
+  if (warp == kMmaWarp) {
+    tmem_alloc_pair(smem_addr(&sm->tmem_base), kTmemCols);
+    tmem_relinquish_pair();
+  }
+  if (warp == kProducerWarp && lane == 0) {
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+  }
+  tc_fence_before();
+  // both CTAs' TMEM is allocated before the first pair MMA
+  cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem = sm->tmem_base;
+  volatile int* abort = &sm->abort;
+  const uint32_t peer_abort = smem_map_rank(smem_addr(&sm->abort), rank ^ 1u);
+
+  if (warp >= kProducerWarp) {
+    regs_dec<kRegsOther>();
+    if ((warp == kProducerWarp || warp == kProducerVWarp) && lane == 0) {
+      // ------------------------------------------------------------ producers
+      const bool is_v = warp == kProducerVWarp;
+      const uint64_t keep = l2_policy_evict_last();
+      const uint64_t once = l2_policy_evict_first();
+      const int depth = is_v ? kStagesV : kStagesK;
+      int gb = 0;  // key blocks loaded so far (all items)
+      int k = 0;
+      bool ok = true;
+      for (int item; ok && (item = pair_id + k * n_pairs) < p.n_items; ++k) {
+        const PairItem it = decode_pair_item(p, item);
+        if (!is_v) {
+          const int qb = k & 1;
+          if (k >= 2 && !mbar_wait_pair(smem_addr(&sm->q_empty[qb]), ((k >> 1) - 1) & 1, abort,
+                                        peer_abort, to, kSitePairProducerQ)) {
+            ok = false;
+            break;
+          }
+          const uint32_t qf = smem_addr(&sm->q_full[qb]);
+          if (leader) mbar_arrive_expect_tx(qf, 2 * kTileBytes);
+          const uint32_t qf0 = smem_map_rank(qf, 0);
+          const int q_row = (it.b * p.Hq + it.hq) * p.S + it.qb2 * kItemRows + rank * kBlockM;
+          const uint32_t q_s = smem_addr(sm->q[qb]);
+          tma_load_2d_pair(q_s, &tm_q, qf0, 0, q_row, once);
+          tma_load_2d_pair(q_s + kPanelBytes, &tm_q, qf0, 64, q_row, once);
+        }
+        const int kv_row = (it.b * p.Hkv + it.g) * p.S;
+        for (int j = 0; j < it.n_blocks; ++j, ++gb) {
+          const int st = gb % depth;
+          const uint32_t empty = smem_addr(is_v ? &sm->v_empty[st] : &sm->k_empty[st]);
+          if (gb >= depth &&
+              !mbar_wait_pair(empty, ((gb / depth) & 1) ^ 1, abort, peer_abort, to,
+                              is_v ? kSitePairProducerV : kSitePairProducerK)) {
+            ok = false;
+            break;
+          }
+          const uint32_t full = smem_addr(is_v ? &sm->v_full[st] : &sm->k_full[st]);
+          if (leader) mbar_arrive_expect_tx(full, 2 * kHalfBytes);
+          const uint32_t full0 = smem_map_rank(full, 0);
+          if (is_v) {
+            // all 128 keys, head-dimension columns [64 rank, 64 rank + 64)
+            tma_load_2d_pair(smem_addr(sm->v[st]), &tm_v, full0, 64 * rank, kv_row + j * kBlockN,
+                             keep);
+          } else {
+            // keys [64 rank, 64 rank + 64) of the block, both column panels
+            const int key_row = kv_row + j * kBlockN + 64 * rank;
+            tma_load_2d_pair(smem_addr(sm->k[st]), &tm_k, full0, 0, key_row, keep);
+            tma_load_2d_pair(smem_addr(sm->k[st]) + kKPanelBytes, &tm_k, full0, 64, key_row, keep);
+          }
+        }
+      }
+      if (*abort) {
+        // copies still in flight land within microseconds; the even CTA's
+        // full barriers count both CTAs' bytes, so it also waits on those
+        if (leader) {
+          if (!is_v && k > 0) drain_wait(smem_addr(&sm->q_full[(k - 1) & 1]), ((k - 1) >> 1) & 1, to);
+          for (int t = (gb > depth ? gb - depth : 0); t < gb; ++t)
+            drain_wait(smem_addr(is_v ? &sm->v_full[t % depth] : &sm->k_full[t % depth]),
+                       (t / depth) & 1, to);
+        } else {
+          pair_sleep_ns(200000);
+        }
+      }
+    } else if (warp == kMmaWarp && lane == 0 && leader) {
+      // ------------------------------------------------------------ MMA issuer
+      // Block sequence g over all items of the pair: S(g) into S[g & 1], then
+      // PV(g - 1) -- so S(g + 1) never waits for the softmax of block g.
+      int g = 0;
+      bool ok = true;
+      bool have_prev = false;
+      int pv_g = 0, pv_k = 0, pv_j = 0, pv_n = 0;
+      auto issue_pv_block = [&]() -> bool {
+        const int st_v = pv_g % kStagesV;
+        if (!mbar_wait_pair(smem_addr(&sm->v_full[st_v]), (pv_g / kStagesV) & 1, abort, peer_abort,
+                            to, kSitePairMmaV))
+          return false;
+        // the epilogue has read O[pv_k & 1] of item pv_k - 2
+        if (pv_j == 0 && pv_k >= 2 &&
+            !mbar_wait_pair(smem_addr(&sm->o_free[pv_k & 1]), ((pv_k >> 1) - 1) & 1, abort,
+                            peer_abort, to, kSitePairMmaO))
+          return false;
+        if (!mbar_wait_pair(smem_addr(&sm->p_full[pv_g & 1]), (pv_g >> 1) & 1, abort, peer_abort,
+                            to, kSitePairMmaP))
+          return false;
+        tc_fence_after();
+        issue_pv_pair(tmem + tmem_o(pv_k & 1), tmem + tmem_s(pv_g & 1), smem_addr(sm->v[st_v]),
+                      pv_j > 0);
+        tc_commit_pair(smem_addr(&sm->pv_done[pv_g & 1]), kBothCtas);
+        tc_commit_pair(smem_addr(&sm->v_empty[st_v]), kBothCtas);
+        if (pv_j == pv_n - 1) tc_commit_pair(smem_addr(&sm->o_done[pv_k & 1]), kBothCtas);
+        return true;
+      };
+      int k = 0;
+      for (int item; ok && (item = pair_id + k * n_pairs) < p.n_items; ++k) {
+        const PairItem it = decode_pair_item(p, item);
+        const int qb = k & 1;
+        if (!mbar_wait_pair(smem_addr(&sm->q_full[qb]), (k >> 1) & 1, abort, peer_abort, to,
+                            kSitePairMmaQ)) {
+          ok = false;
+          break;
+        }
+        for (int j = 0; j < it.n_blocks; ++j, ++g) {
+          const int st_k = g % kStagesK;
+          if (!mbar_wait_pair(smem_addr(&sm->k_full[st_k]), (g / kStagesK) & 1, abort, peer_abort,
+                              to, kSitePairMmaK)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          issue_qk_pair(tmem + tmem_s(g & 1), smem_addr(sm->q[qb]), smem_addr(sm->k[st_k]));
+          tc_commit_pair(smem_addr(&sm->s_full[g & 1]), kBothCtas);
+          tc_commit_pair(smem_addr(&sm->k_empty[st_k]), kBothCtas);
+          if (j == it.n_blocks - 1) tc_commit_pair(smem_addr(&sm->q_empty[qb]), kBothCtas);
+          if (have_prev && !issue_pv_block()) {
+            ok = false;
+            break;
+          }
+          have_prev = true;
+          pv_g = g;
+          pv_k = k;
+          pv_j = j;
+          pv_n = it.n_blocks;
+        }
+      }
+      if (ok && have_prev) issue_pv_block();
+      // every MMA issued must complete before either CTA releases its TMEM
+      tc_commit_pair(smem_addr(&sm->drain), kBothCtas);
+    }
+    __syncwarp();
+    if (warp == kMmaWarp) {
+      // both CTAs: the drain commit has landed (or the wait gave up)
+      if (lane == 0) drain_wait(smem_addr(&sm->drain), 0, to);
+      __syncwarp();
+    }
+  } else if (warp >= kEpilogueWarp0) {
+    // -------------------------------------------------------------- epilogue
+    regs_dec<kRegsEpilogue>();
+    const int r = (warp - kEpilogueWarp0) * 32 + lane;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+    const uint32_t o_free0[2] = {smem_map_rank(smem_addr(&sm->o_free[0]), 0),
+                                 smem_map_rank(smem_addr(&sm->o_free[1]), 0)};
+    const uint32_t item_flag0[2] = {smem_map_rank(smem_addr(&sm->item_flag[0]), 0),
+                                    smem_map_rank(smem_addr(&sm->item_flag[1]), 0)};
+    const uint32_t item_warps0[2] = {smem_map_rank(smem_addr(&sm->item_warps[0]), 0),
+                                     smem_map_rank(smem_addr(&sm->item_warps[1]), 0)};
+    int k = 0;
+    for (int item; (item = pair_id + k * n_pairs) < p.n_items; ++k) {
+      const PairItem it = decode_pair_item(p, item);
+      const int ob = k & 1;
+      bool ok = mbar_wait_pair(smem_addr(&sm->o_done[ob]), (k >> 1) & 1, abort, peer_abort, to,
+                               kSitePairEpilogueO) &&
+                mbar_wait_pair(smem_addr(&sm->stats_ready[ob]), (k >> 1) & 1, abort, peer_abort, to,
+                               kSitePairEpilogueStats);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      const float m_use = sm->stat_m[ob][r];
+      const float l = sm->stat_l[ob][r];
+      mbar_arrive(smem_addr(&sm->stats_free[ob]));
+      bool flag = false;
+      if (rank == 0 || it.half1) {
+        const float inv_l = 1.0f / l;
+        const int row = (it.b * p.Hq + it.hq) * p.S + it.qb2 * kItemRows + rank * kBlockM + r;
+        uint4* orow = reinterpret_cast<uint4*>(p.o + static_cast<size_t>(row) * kHeadDim);
+        float omax = 0.f;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          uint32_t w[16];
+          tmem_ld16(lane_base + tmem_o(ob) + c * 16, w);
+          tmem_wait_ld();
+          reg_dep16(w);
+#pragma unroll
+          for (int v4 = 0; v4 < 2; ++v4) {
+            float f[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              f[e] = __uint_as_float(w[v4 * 8 + e]) * inv_l;
+              omax = fmaxf(omax, fabsf(f[e]));
+            }
+            uint4 pk;
+            pk.x = pack_half2(f[0], f[1]);
+            pk.y = pack_half2(f[2], f[3]);
+            pk.z = pack_half2(f[4], f[5]);
+            pk.w = pack_half2(f[6], f[7]);
+            orow[c * 2 + v4] = pk;
+          }
+        }
+        p.lse[row] = (m_use + log2f(l)) * kLn2;
+        flag = omax >= kRedoThreshold;
+      }
+      // One redo-list entry per item if any row of either CTA needs it: the
+      // 8 epilogue warps of the pair count in on the even CTA's words, and
+      // the last one appends.  This comes before the o_free arrive, so no
+      // warp reaches item k + 2 (whose first PV waits for o_free of item k)
+      // before all 8 have left the parity slot of item k.
+      const bool any = __any_sync(0xffffffffu, flag);
+      if (lane == 0) {
+        if (any) atom_or_cluster(item_flag0[ob], 1u);
+        if (atom_add_cluster(item_warps0[ob], 1u) == 7u) {
+          atom_exch_cluster(item_warps0[ob], 0u);
+          if (atom_exch_cluster(item_flag0[ob], 0u)) {
+            const unsigned int slot = atomicAdd(p.redo, 1u);
+            if (slot < p.redo_capacity)
+              p.redo[kRedoHeaderWords + slot] = static_cast<unsigned int>(item);
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(o_free0[ob]);
+    }
+  } else {
+    // -------------------------------------------------------------- softmax
+    regs_inc<kRegsSoftmax>();
+    const int r = warp * 32 + lane;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    const uint32_t p_full0[2] = {smem_map_rank(smem_addr(&sm->p_full[0]), 0),
+                                 smem_map_rank(smem_addr(&sm->p_full[1]), 0)};
+    const float sc = p.scale_log2;
+    const float2 sc2 = make_float2(sc, sc);
+    int g = 0;
+    int k = 0;
+    for (int item; (item = pair_id + k * n_pairs) < p.n_items; ++k) {
+      const PairItem it = decode_pair_item(p, item);
+      const bool active = rank == 0 || it.half1;
+      const int ob = k & 1;
+      const uint32_t o_t = lane_base + tmem_o(ob);
+      // this CTA's diagonal key block (causal): rows start at 128 (2 qb2 + rank)
+      const int diag = p.causal ? 2 * it.qb2 + static_cast<int>(rank) : (1 << 30);
+      float m_use = -INFINITY;
+      float l = 0.f;
+      bool ok = true;
+      for (int j = 0; j < it.n_blocks; ++j, ++g) {
+        ok = mbar_wait_pair(smem_addr(&sm->s_full[g & 1]), (g >> 1) & 1, abort, peer_abort, to,
+                            kSitePairSoftmaxS);
+        if (!__all_sync(0xffffffffu, ok)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t s_t = lane_base + tmem_s(g & 1);
+        if (active) {
+          uint32_t u[128];
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+            tmem_ld32(s_t + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&u[c * 32]));
+          tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < 4; ++c) reg_dep32(&u[c * 32]);
+          if (j >= diag) {
+            // the diagonal block keeps keys <= row; blocks past it keep none
+            const int lim = j == diag ? r : -1;
+#pragma unroll
+            for (int c = 0; c < 128; ++c)
+              if (c > lim) u[c] = 0xff800000u;  // -inf
+          }
+          float mx8[8];
+#pragma unroll
+          for (int t = 0; t < 8; ++t) mx8[t] = __uint_as_float(u[t]);
+#pragma unroll
+          for (int c = 8; c < 128; c += 16)
+#pragma unroll
+            for (int t = 0; t < 8; ++t)
+              mx8[t] = fmax3(mx8[t], __uint_as_float(u[c + t]), __uint_as_float(u[c + 8 + t]));
+          const float cand = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
+                                   fmaxf(mx8[6], mx8[7])) * sc;
+          if (j == 0) {
+            m_use = cand;
+          } else {
+            const bool grow = cand > m_use + kRescaleLog2;
+            if (__any_sync(0xffffffffu, grow)) {
+              // O[ob] must hold every PV of this item so far: PV(g - 1) may
+              // still be in flight (S(g) was issued before it)
+              ok = mbar_wait_pair(smem_addr(&sm->pv_done[(g - 1) & 1]), ((g - 1) >> 1) & 1, abort,
+                                  peer_abort, to, kSitePairSoftmaxPV);
+              if (!__all_sync(0xffffffffu, ok)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              const float alpha = grow ? ex2_approx(m_use - cand) : 1.0f;
+#pragma unroll 1
+              for (int c = 0; c < 4; ++c) {
+                uint32_t w[32];
+                tmem_ld32(o_t + c * 32, w);
+                tmem_wait_ld();
+                reg_dep32(w);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(__uint_as_float(w[i]) * alpha);
+                tmem_st32(o_t + c * 32, w);
+              }
+              if (grow) {
+                l *= alpha;
+                m_use = cand;
+              }
+            }
+          }
+          // P rounded to fp16 over the first 64 columns of S; l sums exactly
+          // the rounded values
+          const float2 nm2 = make_float2(-m_use, -m_use);
+          float lp[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            uint32_t ph[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const float2 s2 = make_float2(__uint_as_float(u[c * 16 + 2 * i]),
+                                            __uint_as_float(u[c * 16 + 2 * i + 1]));
+              const float2 x2 = __ffma2_rn(s2, sc2, nm2);
+              ph[i] = pack_half2(ex2_approx(x2.x), ex2_approx(x2.y));
+              lp[i & 3] = add_half2_f32(ph[i], lp[i & 3]);
+            }
+            tmem_st8(s_t + c * 8, ph);
+          }
+          l += (lp[0] + lp[1]) + (lp[2] + lp[3]);
+          tmem_wait_st();
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(p_full0[g & 1]);
+      }
+      if (!ok) break;
+      // the epilogue has read the statistics of item k - 2
+      ok = k < 2 || mbar_wait_pair(smem_addr(&sm->stats_free[ob]), ((k >> 1) - 1) & 1, abort,
+                                   peer_abort, to, kSitePairSoftmaxStats);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      sm->stat_m[ob][r] = m_use;
+      sm->stat_l[ob][r] = l;
+      mbar_arrive(smem_addr(&sm->stats_ready[ob]));
+    }
+  }
+
+  tc_fence_before();
+  // every role of both CTAs is done, and the MMAs have drained
+  cluster_sync();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, kTmemCols);
+  }
+}
+
+}  // namespace pair
+}  // namespace attn_b200

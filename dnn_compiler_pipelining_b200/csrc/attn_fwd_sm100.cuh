@@ -468,6 +468,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t w[16];
             tmem_ld16(lane_base + tmem_o_col(x) + c * 16, w);
             tmem_wait_ld();
+            reg_dep16(w);
 #pragma unroll
             for (int v4 = 0; v4 < 2; ++v4) {
               float f[8];
@@ -545,6 +546,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int c = 0; c < 4; ++c)
             tmem_ld32(s_t + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&u[c * 32]));
           tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < 4; ++c) reg_dep32(&u[c * 32]);
           if (j == diag) {
 #pragma unroll
             for (int c = 0; c < 128; ++c)
@@ -573,6 +576,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 uint32_t w[32];
                 tmem_ld32(o_t + c * 32, w);
                 tmem_wait_ld();
+                reg_dep32(w);
 #pragma unroll
                 for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(__uint_as_float(w[i]) * alpha);
                 tmem_st32(o_t + c * 32, w);

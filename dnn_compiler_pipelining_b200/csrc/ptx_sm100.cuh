@@ -188,6 +188,24 @@ __device__ __forceinline__ void tc_commit(uint32_t bar) {
 __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
+
+// tcgen05.ld writes its destination registers asynchronously: they hold the
+// loaded values only after tcgen05.wait::ld.  The compiler does not know
+// that, so after the wait each loaded register is passed through an empty
+// asm that "redefines" it; no read or write of the register can then be
+// scheduled before the wait.
+__device__ __forceinline__ void reg_dep8(uint32_t* r) {
+  asm volatile("" : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
+                    "+r"(r[6]), "+r"(r[7]));
+}
+__device__ __forceinline__ void reg_dep16(uint32_t* r) {
+  reg_dep8(r);
+  reg_dep8(r + 8);
+}
+__device__ __forceinline__ void reg_dep32(uint32_t* r) {
+  reg_dep16(r);
+  reg_dep16(r + 16);
+}
 __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
@@ -426,5 +444,154 @@ __device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {
         "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]),
         "=r"(r[62]), "=r"(r[63])
       : "r"(taddr));
+}
+}  // namespace attn_b200
+
+namespace attn_b200 {
+// --------------------------------------------------------------------------
+// CTA pairs (a 2-CTA cluster on two SMs): one tcgen05.mma.cta_group::2 spans
+// both SMs, M = 256 (each CTA holds 128 rows of A and of the accumulator in
+// its own TMEM, and half of B's N rows in its own shared memory).  Only the
+// even CTA issues MMAs and commits; the odd one supplies its operands.
+// --------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cluster_nctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+  return r;
+}
+// Address of the same shared-memory offset in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t smem_map_rank(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+// Every thread of both CTAs: release own prior writes, wait for the others'.
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" :::
+                   "memory");
+}
+__device__ __forceinline__ void st_cluster_u32(uint32_t caddr, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(caddr), "r"(v) : "memory");
+}
+
+// TMEM for pair MMAs: the same warp index of both CTAs executes these.
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t dst, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+
+// Pair MMAs with compile-time descriptor offsets (16-byte units for shared
+// memory, columns for TMEM), as mma_f16_ss_off / mma_f16_ts_off.
+template <uint32_t kOffA, uint32_t kOffB>
+__device__ __forceinline__ void mma_pair_ss_off(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                                uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b64 da, db;\n\t"
+      "add.s64 da, %1, %5;\n\t"
+      "add.s64 db, %2, %6;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], da, db, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "n"(kOffA), "n"(kOffB)
+      : "memory");
+}
+template <uint32_t kOffA, uint32_t kOffB>
+__device__ __forceinline__ void mma_pair_ts_off(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                                uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b64 db;\n\t.reg .b32 ta;\n\t"
+      "add.u32 ta, %1, %5;\n\t"
+      "add.s64 db, %2, %6;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], [ta], db, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate), "n"(kOffA), "n"(kOffB)
+      : "memory");
+}
+// Arrives once on the barrier at offset `bar` of every CTA in `cta_mask`
+// when all pair MMAs this thread issued before it have completed.
+__device__ __forceinline__ void tc_commit_pair(uint32_t bar, uint16_t cta_mask) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 "
+      "[%0], %1;" ::"r"(bar),
+      "h"(cta_mask)
+      : "memory");
+}
+// Tile load into this CTA's shared memory whose completion (bytes) is
+// counted on `bar`, which may be the even CTA's barrier (no multicast).
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                                 int32_t x, int32_t y, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      ".L2::cache_hint [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y), "l"(policy)
+      : "memory");
+}
+// Atomics on a shared-memory word of any CTA of the cluster.
+__device__ __forceinline__ uint32_t atom_add_cluster(uint32_t caddr, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.acq_rel.cluster.shared::cluster.add.u32 %0, [%1], %2;"
+               : "=r"(old)
+               : "r"(caddr), "r"(v)
+               : "memory");
+  return old;
+}
+__device__ __forceinline__ uint32_t atom_or_cluster(uint32_t caddr, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.acq_rel.cluster.shared::cluster.or.b32 %0, [%1], %2;"
+               : "=r"(old)
+               : "r"(caddr), "r"(v)
+               : "memory");
+  return old;
+}
+__device__ __forceinline__ uint32_t atom_exch_cluster(uint32_t caddr, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.acq_rel.cluster.shared::cluster.exch.b32 %0, [%1], %2;"
+               : "=r"(old)
+               : "r"(caddr), "r"(v)
+               : "memory");
+  return old;
+}
+// Arrive on a barrier of either CTA of the pair.  What the arrive publishes
+// is TMEM contents (ordered by tcgen05.wait + tcgen05.fence before it and
+// tcgen05.fence::after_thread_sync after the wait) or the completion of a
+// read, so CTA-scope release suffices; a cluster-scope release would also
+// drain this thread's outstanding memory traffic to cluster scope, which
+// measured about 1000 cycles per arrive.
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t caddr) {
+  asm volatile("mbarrier.arrive.release.cta.shared::cluster.b64 _, [%0];" ::"r"(caddr)
+               : "memory");
+}
+// As mbar_wait; on running out it also raises the other CTA's abort flag
+// (cluster address `peer_abort`).
+__device__ __forceinline__ bool mbar_wait_pair(uint32_t bar, uint32_t parity, volatile int* abort,
+                                               uint32_t peer_abort, uint64_t timeout_ns,
+                                               uint32_t site) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 32; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (*abort) return false;
+    if (global_timer_ns() - t0 > timeout_ns) {
+      *abort = 1;
+      st_cluster_u32(peer_abort, 1u);
+      atomicOr(&g_attn_status[0], kStatusTimeout);
+      atomicCAS(&g_attn_status[1], 0u, site);
+      return false;
+    }
+  }
 }
 }  // namespace attn_b200
