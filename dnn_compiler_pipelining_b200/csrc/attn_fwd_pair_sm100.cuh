@@ -14,24 +14,29 @@
 // the 128 head-dimension columns of V_j -- so every K/V byte crosses from L2
 // into shared memory once per pair, not once per SM.
 //
-// Each CTA's TMEM (512 columns) holds two S buffers and two O buffers:
-//   S[0] [0,128)  S[1] [128,256)   (key block g of the pair's block
-//   sequence goes to S[g & 1]; P_g, fp16, is written over its first 64
-//   columns)
-//   O[0] [256,384) O[1] [384,512)  (item k accumulates in O[k & 1])
-// With S double-buffered the MMA warp issues S(g+1) before PV(g): the
-// softmax of block g+1 never waits for PV(g), and the tensor core computes
-// S(g+1) while the softmax works on block g.  With O double-buffered the
-// epilogue of item k overlaps item k+1.  Q is double-buffered too, so the
-// next item's Q is in shared memory before its first S.
+// Each CTA's TMEM (512 columns) holds three S buffers and the O accumulator:
+//   S[0] [0,128)  S[1] [128,256)  S[2] [256,384)   (key block g of the
+//   pair's block sequence goes to S[g % 3]; P_g, fp16, is written over its
+//   first 64 columns)
+//   O    [384,512)
+// The MMA warp issues S(g+3) right after PV(g), so the S of the next two
+// blocks is always ready when a softmax warpgroup turns to it.
 //
-// Warp roles (384 threads per CTA):
-//   warps 0-3   softmax (one query row per thread = TMEM lane)
-//   warps 4-7   epilogue: O / l -> fp16, LSE
-//   warp 8      TMA producer of Q (per item) and this CTA's half of K_j
-//   warp 9      MMA issuer (even CTA, one thread); TMEM allocation (both)
-//   warp 10     TMA producer of this CTA's half of V_j
-//   warp 11     idle
+// The softmax runs in two warpgroups that take alternate key blocks (WG0
+// the even blocks g, WG1 the odd ones).  The running row max is handed from
+// block to block through shared memory (m_ready / m_pub); each warpgroup
+// keeps its own partial row sum l relative to the last max it used, and the
+// epilogue combines the two.  While one warpgroup computes the max of its
+// block, the other's exponentials keep the MUFU unit busy.
+//
+// Warp roles (512 threads per CTA):
+//   warps 0-3   softmax warpgroup 0 (one query row per thread = TMEM lane)
+//   warps 4-7   softmax warpgroup 1
+//   warps 8-11  epilogue: O / l -> fp16, LSE
+//   warp 12     TMA producer of Q (per item) and this CTA's half of K_j
+//   warp 13     MMA issuer (even CTA, one thread); TMEM allocation (both)
+//   warp 14     TMA producer of this CTA's half of V_j
+//   warp 15     idle
 //
 // Signals between the two CTAs: the odd CTA's loads complete their bytes
 // on the even CTA's "full" barriers; the even CTA's commits arrive on the
@@ -51,20 +56,21 @@ constexpr int kStagesK = 4;                            // K ring (this CTA's 64 
 constexpr int kStagesV = 4;                            // V ring (this CTA's 64 columns of a block)
 constexpr uint32_t kHalfBytes = kTileBytes / 2;        // 16 KiB
 constexpr uint32_t kKPanelBytes = kHalfBytes / 2;      // 64 keys x 64 columns
-constexpr int kThreads = 384;
-constexpr int kEpilogueWarp0 = 4;
-constexpr int kProducerWarp = 8;
-constexpr int kMmaWarp = 9;
-constexpr int kProducerVWarp = 10;
-constexpr int kRegsSoftmax = 224;
-constexpr int kRegsEpilogue = 96;
-constexpr int kRegsOther = 56;
-static_assert(128 * kRegsSoftmax + 128 * kRegsEpilogue + 128 * kRegsOther <= 65536,
+constexpr int kThreads = 512;
+constexpr int kEpilogueWarp0 = 8;
+constexpr int kProducerWarp = 12;
+constexpr int kMmaWarp = 13;
+constexpr int kProducerVWarp = 14;
+constexpr int kRegsSoftmax = 184;
+constexpr int kRegsEpilogue = 80;
+constexpr int kRegsOther = 64;
+static_assert(256 * kRegsSoftmax + 128 * kRegsEpilogue + 128 * kRegsOther <= 65536,
               "register split exceeds the register file");
 constexpr uint16_t kBothCtas = 0x3;
+constexpr int kSBufs = 3;
 
 __device__ __forceinline__ uint32_t tmem_s(int b) { return static_cast<uint32_t>(b) * 128u; }
-__device__ __forceinline__ uint32_t tmem_o(int b) { return 256u + static_cast<uint32_t>(b) * 128u; }
+constexpr uint32_t kTmemO = 384u;
 
 enum PairWaitSite : uint32_t {
   kSitePairProducerQ = 0x1101,
@@ -89,11 +95,14 @@ struct SharedPair {
   uint8_t q[2][kTileBytes];         // [item parity] this CTA's 128 rows, two 64-column panels
   uint8_t k[kStagesK][kHalfBytes];  // 64 keys x 128 columns, two panels of 8 KiB
   uint8_t v[kStagesV][kHalfBytes];  // 128 keys x 64 columns (one panel)
-  float stat_m[2][kBlockM];         // [item parity][row]
-  float stat_l[2][kBlockM];
+  float stat_m[2][2][kBlockM];      // [item parity][softmax warpgroup][row]
+  float stat_l[2][2][kBlockM];
+  float m_pub[2][kBlockM];          // [block parity][row]: row max after that block
   uint64_t q_full[2], q_empty[2];
   uint64_t k_full[kStagesK], k_empty[kStagesK], v_full[kStagesV], v_empty[kStagesV];
-  uint64_t s_full[2], p_full[2], pv_done[2], o_done[2], o_free[2];
+  uint64_t s_full[kSBufs], p_full[kSBufs];     // [S buffer]
+  uint64_t pv_done[2], m_ready[2];             // [block parity]
+  uint64_t o_done, o_free;
   uint64_t stats_ready[2], stats_free[2];
   uint64_t drain;
   uint32_t tmem_base;
@@ -180,6 +189,37 @@ __device__ __forceinline__ void pair_sleep_ns(uint64_t ns) {
   while (global_timer_ns() - t0 < ns) __nanosleep(1000);
 }
 
+// Cursor over the key blocks of a pair's items, in issue order: item k,
+// block j of n, global block index g.
+struct BlockCursor {
+  int k, j, n, g, item;
+  PairItem it;
+};
+
+__device__ __forceinline__ bool cursor_start(BlockCursor& c, const FwdParams& p, int pair_id,
+                                             int n_pairs) {
+  c.k = 0;
+  c.j = 0;
+  c.g = 0;
+  c.item = pair_id;
+  if (c.item >= p.n_items) return false;
+  c.it = decode_pair_item(p, c.item);
+  c.n = c.it.n_blocks;
+  return true;
+}
+
+__device__ __forceinline__ bool cursor_next(BlockCursor& c, const FwdParams& p, int n_pairs) {
+  ++c.g;
+  if (++c.j < c.n) return true;
+  c.j = 0;
+  ++c.k;
+  c.item += n_pairs;
+  if (c.item >= p.n_items) return false;
+  c.it = decode_pair_item(p, c.item);
+  c.n = c.it.n_blocks;
+  return true;
+}
+
 // The fused pass on CTA pairs (records items for the redo pass exactly as
 // attn_fwd_kernel<0> does).  Launched with 2-CTA clusters; the grid is an
 // even number of CTAs, pair c taking items c, c + pairs, ...
@@ -206,21 +246,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     for (int b = 0; b < 2; ++b) {
       mbar_init(smem_addr(&sm->q_full[b]), 1);
       mbar_init(smem_addr(&sm->q_empty[b]), 1);
-      mbar_init(smem_addr(&sm->s_full[b]), 1);
-      mbar_init(smem_addr(&sm->p_full[b]), 8);   // 4 softmax warps x 2 CTAs
       mbar_init(smem_addr(&sm->pv_done[b]), 1);
-      mbar_init(smem_addr(&sm->o_done[b]), 1);
-      mbar_init(smem_addr(&sm->o_free[b]), 8);   // 4 epilogue warps x 2 CTAs
-      mbar_init(smem_addr(&sm->stats_ready[b]), kBlockM);
+      mbar_init(smem_addr(&sm->m_ready[b]), kBlockM);
+      mbar_init(smem_addr(&sm->stats_ready[b]), 2 * kBlockM);
       mbar_init(smem_addr(&sm->stats_free[b]), kBlockM);
     }
-    for (int s = 0; s < kStagesK; ++s) {
-      mbar_init(smem_addr(&sm->k_full[s]), 1);
-      mbar_init(smem_addr(&sm->k_empty[s]), 1);
+    for (int b = 0; b < kSBufs; ++b) {
+      mbar_init(smem_addr(&sm->s_full[b]), 1);
+      // P of the block in S[b]: 4 softmax warps x 2 CTAs.  Indexed by buffer,
+      // not by warpgroup: a warpgroup may finish two of its blocks before
+      // the MMA thread takes the first (at an item boundary), but block
+      // g + 3 (same buffer) waits for PV(g), so this barrier never runs two
+      // phases ahead of its waiter.
+      mbar_init(smem_addr(&sm->p_full[b]), 8);
     }
-    for (int s = 0; s < kStagesV; ++s) {
-      mbar_init(smem_addr(&sm->v_full[s]), 1);
-      mbar_init(smem_addr(&sm->v_empty[s]), 1);
+    mbar_init(smem_addr(&sm->o_done), 1);
+    mbar_init(smem_addr(&sm->o_free), 8);         // 4 epilogue warps x 2 CTAs
+    for (int st = 0; st < kStagesK; ++st) {
+      mbar_init(smem_addr(&sm->k_full[st]), 1);
+      mbar_init(smem_addr(&sm->k_empty[st]), 1);
+    }
+    for (int st = 0; st < kStagesV; ++st) {
+      mbar_init(smem_addr(&sm->v_full[st]), 1);
+      mbar_init(smem_addr(&sm->v_empty[st]), 1);
     }
     mbar_init(smem_addr(&sm->drain), 1);
     sm->abort = 0;
@@ -316,66 +364,50 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
     } else if (warp == kMmaWarp && lane == 0 && leader) {
       // ------------------------------------------------------------ MMA issuer
-      // Block sequence g over all items of the pair: S(g) into S[g & 1], then
-      // PV(g - 1) -- so S(g + 1) never waits for the softmax of block g.
-      int g = 0;
+      // Two cursors over the block sequence: S(gs) runs three blocks ahead
+      // of PV(gp); S(gp + 3) reuses S[gp % 3] and is issued right after PV(gp).
+      BlockCursor cs, cp;
+      bool s_more = cursor_start(cs, p, pair_id, n_pairs);
+      bool p_more = cursor_start(cp, p, pair_id, n_pairs);
       bool ok = true;
-      bool have_prev = false;
-      int pv_g = 0, pv_k = 0, pv_j = 0, pv_n = 0;
-      auto issue_pv_block = [&]() -> bool {
-        const int st_v = pv_g % kStagesV;
-        if (!mbar_wait_pair(smem_addr(&sm->v_full[st_v]), (pv_g / kStagesV) & 1, abort, peer_abort,
-                            to, kSitePairMmaV))
+      auto issue_s = [&]() -> bool {
+        const int qb = cs.k & 1;
+        if (cs.j == 0 && !mbar_wait_pair(smem_addr(&sm->q_full[qb]), (cs.k >> 1) & 1, abort,
+                                         peer_abort, to, kSitePairMmaQ))
           return false;
-        // the epilogue has read O[pv_k & 1] of item pv_k - 2
-        if (pv_j == 0 && pv_k >= 2 &&
-            !mbar_wait_pair(smem_addr(&sm->o_free[pv_k & 1]), ((pv_k >> 1) - 1) & 1, abort,
-                            peer_abort, to, kSitePairMmaO))
-          return false;
-        if (!mbar_wait_pair(smem_addr(&sm->p_full[pv_g & 1]), (pv_g >> 1) & 1, abort, peer_abort,
-                            to, kSitePairMmaP))
+        const int st_k = cs.g % kStagesK;
+        if (!mbar_wait_pair(smem_addr(&sm->k_full[st_k]), (cs.g / kStagesK) & 1, abort, peer_abort,
+                            to, kSitePairMmaK))
           return false;
         tc_fence_after();
-        issue_pv_pair(tmem + tmem_o(pv_k & 1), tmem + tmem_s(pv_g & 1), smem_addr(sm->v[st_v]),
-                      pv_j > 0);
-        tc_commit_pair(smem_addr(&sm->pv_done[pv_g & 1]), kBothCtas);
-        tc_commit_pair(smem_addr(&sm->v_empty[st_v]), kBothCtas);
-        if (pv_j == pv_n - 1) tc_commit_pair(smem_addr(&sm->o_done[pv_k & 1]), kBothCtas);
+        issue_qk_pair(tmem + tmem_s(cs.g % kSBufs), smem_addr(sm->q[qb]), smem_addr(sm->k[st_k]));
+        tc_commit_pair(smem_addr(&sm->s_full[cs.g % kSBufs]), kBothCtas);
+        tc_commit_pair(smem_addr(&sm->k_empty[st_k]), kBothCtas);
+        if (cs.j == cs.n - 1) tc_commit_pair(smem_addr(&sm->q_empty[qb]), kBothCtas);
+        s_more = cursor_next(cs, p, n_pairs);
         return true;
       };
-      int k = 0;
-      for (int item; ok && (item = pair_id + k * n_pairs) < p.n_items; ++k) {
-        const PairItem it = decode_pair_item(p, item);
-        const int qb = k & 1;
-        if (!mbar_wait_pair(smem_addr(&sm->q_full[qb]), (k >> 1) & 1, abort, peer_abort, to,
-                            kSitePairMmaQ)) {
-          ok = false;
-          break;
-        }
-        for (int j = 0; j < it.n_blocks; ++j, ++g) {
-          const int st_k = g % kStagesK;
-          if (!mbar_wait_pair(smem_addr(&sm->k_full[st_k]), (g / kStagesK) & 1, abort, peer_abort,
-                              to, kSitePairMmaK)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          issue_qk_pair(tmem + tmem_s(g & 1), smem_addr(sm->q[qb]), smem_addr(sm->k[st_k]));
-          tc_commit_pair(smem_addr(&sm->s_full[g & 1]), kBothCtas);
-          tc_commit_pair(smem_addr(&sm->k_empty[st_k]), kBothCtas);
-          if (j == it.n_blocks - 1) tc_commit_pair(smem_addr(&sm->q_empty[qb]), kBothCtas);
-          if (have_prev && !issue_pv_block()) {
-            ok = false;
-            break;
-          }
-          have_prev = true;
-          pv_g = g;
-          pv_k = k;
-          pv_j = j;
-          pv_n = it.n_blocks;
-        }
+      for (int i = 0; ok && s_more && i < kSBufs; ++i) ok = issue_s();
+      while (ok && p_more) {
+        const int st_v = cp.g % kStagesV;
+        // the epilogue has read O of the previous item
+        ok = (cp.j != 0 || cp.k == 0 ||
+              mbar_wait_pair(smem_addr(&sm->o_free), (cp.k - 1) & 1, abort, peer_abort, to,
+                             kSitePairMmaO)) &&
+             mbar_wait_pair(smem_addr(&sm->v_full[st_v]), (cp.g / kStagesV) & 1, abort, peer_abort,
+                            to, kSitePairMmaV) &&
+             mbar_wait_pair(smem_addr(&sm->p_full[cp.g % kSBufs]), (cp.g / kSBufs) & 1, abort,
+                            peer_abort, to, kSitePairMmaP);
+        if (!ok) break;
+        tc_fence_after();
+        issue_pv_pair(tmem + kTmemO, tmem + tmem_s(cp.g % kSBufs), smem_addr(sm->v[st_v]),
+                      cp.j > 0);
+        tc_commit_pair(smem_addr(&sm->pv_done[cp.g & 1]), kBothCtas);
+        tc_commit_pair(smem_addr(&sm->v_empty[st_v]), kBothCtas);
+        if (cp.j == cp.n - 1) tc_commit_pair(smem_addr(&sm->o_done), kBothCtas);
+        p_more = cursor_next(cp, p, n_pairs);
+        if (s_more) ok = issue_s();
       }
-      if (ok && have_prev) issue_pv_block();
       // every MMA issued must complete before either CTA releases its TMEM
       tc_commit_pair(smem_addr(&sm->drain), kBothCtas);
     }
@@ -390,8 +422,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     regs_dec<kRegsEpilogue>();
     const int r = (warp - kEpilogueWarp0) * 32 + lane;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
-    const uint32_t o_free0[2] = {smem_map_rank(smem_addr(&sm->o_free[0]), 0),
-                                 smem_map_rank(smem_addr(&sm->o_free[1]), 0)};
+    const uint32_t o_free0 = smem_map_rank(smem_addr(&sm->o_free), 0);
     const uint32_t item_flag0[2] = {smem_map_rank(smem_addr(&sm->item_flag[0]), 0),
                                     smem_map_rank(smem_addr(&sm->item_flag[1]), 0)};
     const uint32_t item_warps0[2] = {smem_map_rank(smem_addr(&sm->item_warps[0]), 0),
@@ -399,18 +430,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     int k = 0;
     for (int item; (item = pair_id + k * n_pairs) < p.n_items; ++k) {
       const PairItem it = decode_pair_item(p, item);
-      const int ob = k & 1;
-      bool ok = mbar_wait_pair(smem_addr(&sm->o_done[ob]), (k >> 1) & 1, abort, peer_abort, to,
+      const int ib = k & 1;
+      bool ok = mbar_wait_pair(smem_addr(&sm->o_done), k & 1, abort, peer_abort, to,
                                kSitePairEpilogueO) &&
-                mbar_wait_pair(smem_addr(&sm->stats_ready[ob]), (k >> 1) & 1, abort, peer_abort, to,
+                mbar_wait_pair(smem_addr(&sm->stats_ready[ib]), (k >> 1) & 1, abort, peer_abort, to,
                                kSitePairEpilogueStats);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
-      const float m_use = sm->stat_m[ob][r];
-      const float l = sm->stat_l[ob][r];
-      mbar_arrive(smem_addr(&sm->stats_free[ob]));
+      // the two warpgroups' partial sums, each relative to the last max it used
+      const float m0 = sm->stat_m[ib][0][r], l0 = sm->stat_l[ib][0][r];
+      const float m1 = sm->stat_m[ib][1][r], l1 = sm->stat_l[ib][1][r];
+      mbar_arrive(smem_addr(&sm->stats_free[ib]));
       bool flag = false;
       if (rank == 0 || it.half1) {
+        const float m_use = fmaxf(m0, m1);
+        const float l = (l0 > 0.f ? l0 * ex2_approx(m0 - m_use) : 0.f) +
+                        (l1 > 0.f ? l1 * ex2_approx(m1 - m_use) : 0.f);
         const float inv_l = 1.0f / l;
         const int row = (it.b * p.Hq + it.hq) * p.S + it.qb2 * kItemRows + rank * kBlockM + r;
         uint4* orow = reinterpret_cast<uint4*>(p.o + static_cast<size_t>(row) * kHeadDim);
@@ -418,7 +453,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
           uint32_t w[16];
-          tmem_ld16(lane_base + tmem_o(ob) + c * 16, w);
+          tmem_ld16(lane_base + kTmemO + c * 16, w);
           tmem_wait_ld();
           reg_dep16(w);
 #pragma unroll
@@ -443,14 +478,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       // One redo-list entry per item if any row of either CTA needs it: the
       // 8 epilogue warps of the pair count in on the even CTA's words, and
       // the last one appends.  This comes before the o_free arrive, so no
-      // warp reaches item k + 2 (whose first PV waits for o_free of item k)
-      // before all 8 have left the parity slot of item k.
+      // warp reaches item k + 2 (whose first PV waits for o_free of item
+      // k + 1) before all 8 have left the parity slot of item k.
       const bool any = __any_sync(0xffffffffu, flag);
       if (lane == 0) {
-        if (any) atom_or_cluster(item_flag0[ob], 1u);
-        if (atom_add_cluster(item_warps0[ob], 1u) == 7u) {
-          atom_exch_cluster(item_warps0[ob], 0u);
-          if (atom_exch_cluster(item_flag0[ob], 0u)) {
+        if (any) atom_or_cluster(item_flag0[ib], 1u);
+        if (atom_add_cluster(item_warps0[ib], 1u) == 7u) {
+          atom_exch_cluster(item_warps0[ib], 0u);
+          if (atom_exch_cluster(item_flag0[ib], 0u)) {
             const unsigned int slot = atomicAdd(p.redo, 1u);
             if (slot < p.redo_capacity)
               p.redo[kRedoHeaderWords + slot] = static_cast<unsigned int>(item);
@@ -459,40 +494,43 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(o_free0[ob]);
+      if (lane == 0) mbar_arrive_cluster(o_free0);
     }
   } else {
     // -------------------------------------------------------------- softmax
     regs_inc<kRegsSoftmax>();
-    const int r = warp * 32 + lane;
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-    const uint32_t p_full0[2] = {smem_map_rank(smem_addr(&sm->p_full[0]), 0),
-                                 smem_map_rank(smem_addr(&sm->p_full[1]), 0)};
+    const int wg = warp >> 2;  // this warpgroup takes the blocks g with g % 2 == wg
+    const int r = (warp & 3) * 32 + lane;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+    const uint32_t o_t = lane_base + kTmemO;
+    const uint32_t p_full0[kSBufs] = {smem_map_rank(smem_addr(&sm->p_full[0]), 0),
+                                      smem_map_rank(smem_addr(&sm->p_full[1]), 0),
+                                      smem_map_rank(smem_addr(&sm->p_full[2]), 0)};
     const float sc = p.scale_log2;
     const float2 sc2 = make_float2(sc, sc);
-    int g = 0;
+    int g = 0;  // global block index (all items of the pair)
     int k = 0;
-    for (int item; (item = pair_id + k * n_pairs) < p.n_items; ++k) {
+    bool ok = true;
+    for (int item; ok && (item = pair_id + k * n_pairs) < p.n_items; ++k) {
       const PairItem it = decode_pair_item(p, item);
       const bool active = rank == 0 || it.half1;
-      const int ob = k & 1;
-      const uint32_t o_t = lane_base + tmem_o(ob);
       // this CTA's diagonal key block (causal): rows start at 128 (2 qb2 + rank)
       const int diag = p.causal ? 2 * it.qb2 + static_cast<int>(rank) : (1 << 30);
-      float m_use = -INFINITY;
+      float m_ref = -INFINITY;  // the max this warpgroup's l is relative to
       float l = 0.f;
-      bool ok = true;
       for (int j = 0; j < it.n_blocks; ++j, ++g) {
-        ok = mbar_wait_pair(smem_addr(&sm->s_full[g & 1]), (g >> 1) & 1, abort, peer_abort, to,
-                            kSitePairSoftmaxS);
+        if ((g & 1) != wg) continue;
+        ok = mbar_wait_pair(smem_addr(&sm->s_full[g % kSBufs]), (g / kSBufs) & 1, abort, peer_abort,
+                            to, kSitePairSoftmaxS);
         if (!__all_sync(0xffffffffu, ok)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t s_t = lane_base + tmem_s(g & 1);
+        const uint32_t s_t = lane_base + tmem_s(g % kSBufs);
+        uint32_t u[128];
+        float cand = -INFINITY;
         if (active) {
-          uint32_t u[128];
 #pragma unroll
           for (int c = 0; c < 4; ++c)
             tmem_ld32(s_t + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&u[c * 32]));
@@ -506,46 +544,69 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             for (int c = 0; c < 128; ++c)
               if (c > lim) u[c] = 0xff800000u;  // -inf
           }
+          // row max: 8 independent chains (chain t takes columns t, t + 8,
+          // ..., t + 120) of 3-input max, then a tree
           float mx8[8];
 #pragma unroll
-          for (int t = 0; t < 8; ++t) mx8[t] = __uint_as_float(u[t]);
+          for (int t = 0; t < 8; ++t)
+            mx8[t] = fmax3(__uint_as_float(u[t]), __uint_as_float(u[8 + t]),
+                           __uint_as_float(u[16 + t]));
 #pragma unroll
-          for (int c = 8; c < 128; c += 16)
+          for (int c = 24; c < 120; c += 16)
 #pragma unroll
             for (int t = 0; t < 8; ++t)
               mx8[t] = fmax3(mx8[t], __uint_as_float(u[c + t]), __uint_as_float(u[c + 8 + t]));
-          const float cand = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
-                                   fmaxf(mx8[6], mx8[7])) * sc;
-          if (j == 0) {
-            m_use = cand;
-          } else {
-            const bool grow = cand > m_use + kRescaleLog2;
-            if (__any_sync(0xffffffffu, grow)) {
-              // O[ob] must hold every PV of this item so far: PV(g - 1) may
-              // still be in flight (S(g) was issued before it)
-              ok = mbar_wait_pair(smem_addr(&sm->pv_done[(g - 1) & 1]), ((g - 1) >> 1) & 1, abort,
-                                  peer_abort, to, kSitePairSoftmaxPV);
-              if (!__all_sync(0xffffffffu, ok)) {
-                ok = false;
-                break;
-              }
-              tc_fence_after();
-              const float alpha = grow ? ex2_approx(m_use - cand) : 1.0f;
-#pragma unroll 1
-              for (int c = 0; c < 4; ++c) {
-                uint32_t w[32];
-                tmem_ld32(o_t + c * 32, w);
-                tmem_wait_ld();
-                reg_dep32(w);
 #pragma unroll
-                for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(__uint_as_float(w[i]) * alpha);
-                tmem_st32(o_t + c * 32, w);
-              }
-              if (grow) {
-                l *= alpha;
-                m_use = cand;
-              }
+          for (int t = 0; t < 8; ++t) mx8[t] = fmaxf(mx8[t], __uint_as_float(u[120 + t]));
+          cand = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
+                       fmaxf(mx8[6], mx8[7])) * sc;
+        }
+        // the row max after block g - 1 (the other warpgroup's block; for
+        // the first block of an item it belongs to the previous item and
+        // is not used, but every phase is waited on)
+        float m_prev = -INFINITY;
+        if (g > 0) {
+          ok = mbar_wait_pair(smem_addr(&sm->m_ready[(g - 1) & 1]), ((g - 1) >> 1) & 1, abort,
+                              peer_abort, to, kSitePairSoftmaxS);
+          if (!__all_sync(0xffffffffu, ok)) {
+            ok = false;
+            break;
+          }
+          if (j > 0) m_prev = sm->m_pub[(g - 1) & 1][r];
+        }
+        // lazy rescaling: the reference max moves only when the row max
+        // grows by more than 2^kRescaleLog2 (the first block sets it)
+        const bool grow = j == 0 || cand > m_prev + kRescaleLog2;
+        const float m_use = grow ? cand : m_prev;
+        sm->m_pub[g & 1][r] = m_use;
+        mbar_arrive(smem_addr(&sm->m_ready[g & 1]));
+        if (active) {
+          if (j > 0 && __any_sync(0xffffffffu, grow)) {
+            // O must hold every PV of this item so far: PV(g - 1) may still
+            // be in flight
+            ok = mbar_wait_pair(smem_addr(&sm->pv_done[(g - 1) & 1]), ((g - 1) >> 1) & 1, abort,
+                                peer_abort, to, kSitePairSoftmaxPV);
+            if (!__all_sync(0xffffffffu, ok)) {
+              ok = false;
+              break;
             }
+            tc_fence_after();
+            const float alpha = grow ? ex2_approx(m_prev - cand) : 1.0f;
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+              uint32_t w[32];
+              tmem_ld32(o_t + c * 32, w);
+              tmem_wait_ld();
+              reg_dep32(w);
+#pragma unroll
+              for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(__uint_as_float(w[i]) * alpha);
+              tmem_st32(o_t + c * 32, w);
+            }
+          }
+          // this warpgroup's partial sum follows the reference max
+          if (m_use != m_ref) {
+            l = (l > 0.f) ? l * ex2_approx(m_ref - m_use) : 0.f;
+            m_ref = m_use;
           }
           // P rounded to fp16 over the first 64 columns of S; l sums exactly
           // the rounded values
@@ -569,16 +630,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(p_full0[g & 1]);
+        if (lane == 0) mbar_arrive_cluster(p_full0[g % kSBufs]);
       }
       if (!ok) break;
       // the epilogue has read the statistics of item k - 2
-      ok = k < 2 || mbar_wait_pair(smem_addr(&sm->stats_free[ob]), ((k >> 1) - 1) & 1, abort,
+      ok = k < 2 || mbar_wait_pair(smem_addr(&sm->stats_free[k & 1]), ((k >> 1) - 1) & 1, abort,
                                    peer_abort, to, kSitePairSoftmaxStats);
       if (!__all_sync(0xffffffffu, ok)) break;
-      sm->stat_m[ob][r] = m_use;
-      sm->stat_l[ob][r] = l;
-      mbar_arrive(smem_addr(&sm->stats_ready[ob]));
+      sm->stat_m[k & 1][wg][r] = m_ref;
+      sm->stat_l[k & 1][wg][r] = l;
+      mbar_arrive(smem_addr(&sm->stats_ready[k & 1]));
     }
   }
 

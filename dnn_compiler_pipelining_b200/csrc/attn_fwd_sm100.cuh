@@ -553,15 +553,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int c = 0; c < 128; ++c)
               if (c > r) u[c] = 0xff800000u;  // -inf
           }
-          // row max: 8 independent chains of 3-input max, then a tree
+          // row max: 8 independent chains (chain t takes columns t, t + 8,
+          // ..., t + 120) of 3-input max, then a tree
           float mx8[8];
 #pragma unroll
-          for (int t = 0; t < 8; ++t) mx8[t] = __uint_as_float(u[t]);
+          for (int t = 0; t < 8; ++t)
+            mx8[t] = fmax3(__uint_as_float(u[t]), __uint_as_float(u[8 + t]),
+                           __uint_as_float(u[16 + t]));
 #pragma unroll
-          for (int c = 8; c < 128; c += 16)
+          for (int c = 24; c < 120; c += 16)
 #pragma unroll
             for (int t = 0; t < 8; ++t)
               mx8[t] = fmax3(mx8[t], __uint_as_float(u[c + t]), __uint_as_float(u[c + 8 + t]));
+#pragma unroll
+          for (int t = 0; t < 8; ++t) mx8[t] = fmaxf(mx8[t], __uint_as_float(u[120 + t]));
           const float cand = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
                                    fmaxf(mx8[6], mx8[7])) * sc;
           if (j == 0) {
