@@ -71,6 +71,12 @@ unsigned int* redo_list(int dev, cudaStream_t stream) {
   return static_cast<unsigned int*>(ptr);
 }
 
+// Which kernel runs the fused pass: the single-CTA kernel (attn_fwd_kernel<0>)
+// or the CTA-pair kernel (pair::attn_fwd_pair_kernel), which computes the
+// same items and passes the same parity tests but measured slower on B200
+// (793 vs 1003 TFLOP/s at B=64, S=8192, causal).
+constexpr bool kPairFusedPass = false;
+
 size_t fwd_smem_bytes() { return sizeof(SharedFwd); }  // the kernel checks 1 KiB alignment
 size_t pair_smem_bytes() { return sizeof(pair::SharedPair); }
 
@@ -103,16 +109,19 @@ attn_status device_setup(int* dev_out) {
         cudaFuncSetAttribute(pair::attn_fwd_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(pair_smem_bytes())) != cudaSuccess)
       return ATTN_ERR_CUDA;
-    // a persistent grid of as many CTA pairs as can be resident together
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(2 * (g_dev_sms[dev] / 2));
-    cfg.blockDim = dim3(pair::kThreads);
-    cfg.dynamicSmemBytes = pair_smem_bytes();
-    int pairs = 0;
-    if (cudaOccupancyMaxActiveClusters(&pairs, pair::attn_fwd_pair_kernel, &cfg) != cudaSuccess ||
-        pairs < 1)
-      return ATTN_ERR_CUDA;
-    g_dev_pairs[dev] = pairs;
+    if (kPairFusedPass) {
+      // a persistent grid of as many CTA pairs as can be resident together
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(2 * (g_dev_sms[dev] / 2));
+      cfg.blockDim = dim3(pair::kThreads);
+      cfg.dynamicSmemBytes = pair_smem_bytes();
+      int pairs = 0;
+      if (cudaOccupancyMaxActiveClusters(&pairs, pair::attn_fwd_pair_kernel, &cfg) !=
+              cudaSuccess ||
+          pairs < 1)
+        return ATTN_ERR_CUDA;
+      g_dev_pairs[dev] = pairs;
+    }
     g_dev_state[dev].store(1, std::memory_order_release);
   }
   return g_dev_state[dev].load() == 1 ? ATTN_OK : ATTN_ERR_UNSUPPORTED;
@@ -163,11 +172,6 @@ bool encode_call_maps(CallMaps* m, const void* q, const void* k, const void* v, 
   return encode_rows_map(&m->q, q, q_rows) && encode_rows_map(&m->k, k, kv_rows) &&
          encode_rows_map(&m->k_half, k, kv_rows, kBlockM / 2) && encode_rows_map(&m->v, v, kv_rows);
 }
-
-// Which kernel runs the fused pass: the single-CTA kernel (attn_fwd_kernel<0>)
-// or the CTA-pair kernel (pair::attn_fwd_pair_kernel), which computes the
-// same items.
-constexpr bool kPairFusedPass = false;
 
 // The fused pass over every item, then the hi+lo pass over the items it
 // listed.

@@ -34,9 +34,13 @@
 //   warps 4-7   softmax warpgroup 1
 //   warps 8-11  epilogue: O / l -> fp16, LSE
 //   warp 12     TMA producer of Q (per item) and this CTA's half of K_j
-//   warp 13     MMA issuer (even CTA, one thread); TMEM allocation (both)
+//   warp 13     S = Q K^T issuer (even CTA, one thread); TMEM allocation (both)
 //   warp 14     TMA producer of this CTA's half of V_j
-//   warp 15     idle
+//   warp 15     O += P V issuer (even CTA, one thread)
+// Two issuing threads keep the tensor core fed: a single thread waiting on
+// K, V and P and issuing 16 MMAs and their commits per block measured about
+// 2.6x the 1024 cycles the MMAs themselves take.  S(g + 3) overwrites the S
+// buffer of block g, so the S issuer waits for PV(g) to complete (s_free).
 //
 // Signals between the two CTAs: the odd CTA's loads complete their bytes
 // on the even CTA's "full" barriers; the even CTA's commits arrive on the
@@ -61,6 +65,7 @@ constexpr int kEpilogueWarp0 = 8;
 constexpr int kProducerWarp = 12;
 constexpr int kMmaWarp = 13;
 constexpr int kProducerVWarp = 14;
+constexpr int kMmaPvWarp = 15;
 constexpr int kRegsSoftmax = 184;
 constexpr int kRegsEpilogue = 80;
 constexpr int kRegsOther = 64;
@@ -68,6 +73,9 @@ static_assert(256 * kRegsSoftmax + 128 * kRegsEpilogue + 128 * kRegsOther <= 655
               "register split exceeds the register file");
 constexpr uint16_t kBothCtas = 0x3;
 constexpr int kSBufs = 3;
+// Of every 8 column pairs, how many take 2^x from the FMA-pipe polynomial
+// (exp2_poly2) instead of the MUFU unit.
+constexpr int kPairEmuPairs = 0;
 
 __device__ __forceinline__ uint32_t tmem_s(int b) { return static_cast<uint32_t>(b) * 128u; }
 constexpr uint32_t kTmemO = 384u;
@@ -81,6 +89,7 @@ enum PairWaitSite : uint32_t {
   kSitePairMmaV = 0x1203,
   kSitePairMmaP = 0x1204,
   kSitePairMmaO = 0x1205,
+  kSitePairMmaS = 0x1206,
   kSitePairSoftmaxS = 0x1301,
   kSitePairSoftmaxStats = 0x1302,
   kSitePairSoftmaxPV = 0x1303,
@@ -100,7 +109,7 @@ struct SharedPair {
   float m_pub[2][kBlockM];          // [block parity][row]: row max after that block
   uint64_t q_full[2], q_empty[2];
   uint64_t k_full[kStagesK], k_empty[kStagesK], v_full[kStagesV], v_empty[kStagesV];
-  uint64_t s_full[kSBufs], p_full[kSBufs];     // [S buffer]
+  uint64_t s_full[kSBufs], p_full[kSBufs], s_free[kSBufs];  // [S buffer]
   uint64_t pv_done[2], m_ready[2];             // [block parity]
   uint64_t o_done, o_free;
   uint64_t stats_ready[2], stats_free[2];
@@ -259,6 +268,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       // g + 3 (same buffer) waits for PV(g), so this barrier never runs two
       // phases ahead of its waiter.
       mbar_init(smem_addr(&sm->p_full[b]), 8);
+      mbar_init(smem_addr(&sm->s_free[b]), 1);
     }
     mbar_init(smem_addr(&sm->o_done), 1);
     mbar_init(smem_addr(&sm->o_free), 8);         // 4 epilogue warps x 2 CTAs
@@ -270,7 +280,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       mbar_init(smem_addr(&sm->v_full[st]), 1);
       mbar_init(smem_addr(&sm->v_empty[st]), 1);
     }
-    mbar_init(smem_addr(&sm->drain), 1);
+    mbar_init(smem_addr(&sm->drain), 2);  // one commit per issuing thread
     sm->abort = 0;
     sm->item_flag[0] = sm->item_flag[1] = 0;
     sm->item_warps[0] = sm->item_warps[1] = 0;
@@ -363,52 +373,56 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
       }
     } else if (warp == kMmaWarp && lane == 0 && leader) {
-      // ------------------------------------------------------------ MMA issuer
-      // Two cursors over the block sequence: S(gs) runs three blocks ahead
-      // of PV(gp); S(gp + 3) reuses S[gp % 3] and is issued right after PV(gp).
-      BlockCursor cs, cp;
-      bool s_more = cursor_start(cs, p, pair_id, n_pairs);
-      bool p_more = cursor_start(cp, p, pair_id, n_pairs);
-      bool ok = true;
-      auto issue_s = [&]() -> bool {
+      // ---------------------------------------------------------- S issuer
+      BlockCursor cs;
+      bool more = cursor_start(cs, p, pair_id, n_pairs);
+      while (more) {
         const int qb = cs.k & 1;
-        if (cs.j == 0 && !mbar_wait_pair(smem_addr(&sm->q_full[qb]), (cs.k >> 1) & 1, abort,
-                                         peer_abort, to, kSitePairMmaQ))
-          return false;
+        const int sb = cs.g % kSBufs;
         const int st_k = cs.g % kStagesK;
-        if (!mbar_wait_pair(smem_addr(&sm->k_full[st_k]), (cs.g / kStagesK) & 1, abort, peer_abort,
-                            to, kSitePairMmaK))
-          return false;
-        tc_fence_after();
-        issue_qk_pair(tmem + tmem_s(cs.g % kSBufs), smem_addr(sm->q[qb]), smem_addr(sm->k[st_k]));
-        tc_commit_pair(smem_addr(&sm->s_full[cs.g % kSBufs]), kBothCtas);
-        tc_commit_pair(smem_addr(&sm->k_empty[st_k]), kBothCtas);
-        if (cs.j == cs.n - 1) tc_commit_pair(smem_addr(&sm->q_empty[qb]), kBothCtas);
-        s_more = cursor_next(cs, p, n_pairs);
-        return true;
-      };
-      for (int i = 0; ok && s_more && i < kSBufs; ++i) ok = issue_s();
-      while (ok && p_more) {
-        const int st_v = cp.g % kStagesV;
-        // the epilogue has read O of the previous item
-        ok = (cp.j != 0 || cp.k == 0 ||
-              mbar_wait_pair(smem_addr(&sm->o_free), (cp.k - 1) & 1, abort, peer_abort, to,
-                             kSitePairMmaO)) &&
-             mbar_wait_pair(smem_addr(&sm->v_full[st_v]), (cp.g / kStagesV) & 1, abort, peer_abort,
-                            to, kSitePairMmaV) &&
-             mbar_wait_pair(smem_addr(&sm->p_full[cp.g % kSBufs]), (cp.g / kSBufs) & 1, abort,
-                            peer_abort, to, kSitePairMmaP);
+        // Q of a new item; the S buffer (PV of block g - 3 has read its P); K_j
+        const bool ok =
+            (cs.j != 0 || mbar_wait_pair(smem_addr(&sm->q_full[qb]), (cs.k >> 1) & 1, abort,
+                                         peer_abort, to, kSitePairMmaQ)) &&
+            (cs.g < kSBufs || mbar_wait_pair(smem_addr(&sm->s_free[sb]), ((cs.g / kSBufs) - 1) & 1,
+                                             abort, peer_abort, to, kSitePairMmaS)) &&
+            mbar_wait_pair(smem_addr(&sm->k_full[st_k]), (cs.g / kStagesK) & 1, abort, peer_abort,
+                           to, kSitePairMmaK);
         if (!ok) break;
         tc_fence_after();
-        issue_pv_pair(tmem + kTmemO, tmem + tmem_s(cp.g % kSBufs), smem_addr(sm->v[st_v]),
-                      cp.j > 0);
-        tc_commit_pair(smem_addr(&sm->pv_done[cp.g & 1]), kBothCtas);
-        tc_commit_pair(smem_addr(&sm->v_empty[st_v]), kBothCtas);
-        if (cp.j == cp.n - 1) tc_commit_pair(smem_addr(&sm->o_done), kBothCtas);
-        p_more = cursor_next(cp, p, n_pairs);
-        if (s_more) ok = issue_s();
+        issue_qk_pair(tmem + tmem_s(sb), smem_addr(sm->q[qb]), smem_addr(sm->k[st_k]));
+        tc_commit_pair(smem_addr(&sm->s_full[sb]), kBothCtas);
+        tc_commit_pair(smem_addr(&sm->k_empty[st_k]), kBothCtas);
+        if (cs.j == cs.n - 1) tc_commit_pair(smem_addr(&sm->q_empty[qb]), kBothCtas);
+        more = cursor_next(cs, p, n_pairs);
       }
       // every MMA issued must complete before either CTA releases its TMEM
+      tc_commit_pair(smem_addr(&sm->drain), kBothCtas);
+    } else if (warp == kMmaPvWarp && lane == 0 && leader) {
+      // --------------------------------------------------------- PV issuer
+      BlockCursor cp;
+      bool more = cursor_start(cp, p, pair_id, n_pairs);
+      while (more) {
+        const int st_v = cp.g % kStagesV;
+        const int sb = cp.g % kSBufs;
+        // the epilogue has read O of the previous item; V_j; P of this block
+        const bool ok =
+            (cp.j != 0 || cp.k == 0 ||
+             mbar_wait_pair(smem_addr(&sm->o_free), (cp.k - 1) & 1, abort, peer_abort, to,
+                            kSitePairMmaO)) &&
+            mbar_wait_pair(smem_addr(&sm->v_full[st_v]), (cp.g / kStagesV) & 1, abort, peer_abort,
+                           to, kSitePairMmaV) &&
+            mbar_wait_pair(smem_addr(&sm->p_full[sb]), (cp.g / kSBufs) & 1, abort, peer_abort, to,
+                           kSitePairMmaP);
+        if (!ok) break;
+        tc_fence_after();
+        issue_pv_pair(tmem + kTmemO, tmem + tmem_s(sb), smem_addr(sm->v[st_v]), cp.j > 0);
+        tc_commit_pair(smem_addr(&sm->pv_done[cp.g & 1]), kBothCtas);
+        tc_commit_pair(smem_addr(&sm->v_empty[st_v]), kBothCtas);
+        tc_commit_pair(smem_addr(&sm->s_free[sb]), 0x1);
+        if (cp.j == cp.n - 1) tc_commit_pair(smem_addr(&sm->o_done), kBothCtas);
+        more = cursor_next(cp, p, n_pairs);
+      }
       tc_commit_pair(smem_addr(&sm->drain), kBothCtas);
     }
     __syncwarp();
@@ -620,7 +634,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
               const float2 s2 = make_float2(__uint_as_float(u[c * 16 + 2 * i]),
                                             __uint_as_float(u[c * 16 + 2 * i + 1]));
               const float2 x2 = __ffma2_rn(s2, sc2, nm2);
-              ph[i] = pack_half2(ex2_approx(x2.x), ex2_approx(x2.y));
+              if (i < kPairEmuPairs) {
+                const float2 e2 = exp2_poly2(x2);
+                ph[i] = pack_half2(e2.x, e2.y);
+              } else {
+                ph[i] = pack_half2(ex2_approx(x2.x), ex2_approx(x2.y));
+              }
               lp[i & 3] = add_half2_f32(ph[i], lp[i & 3]);
             }
             tmem_st8(s_t + c * 8, ph);
