@@ -149,7 +149,6 @@ attn_status validate_sizes(int B, int Hq, int Hkv, int S, int D) {
   if (B < 1 || Hq < 1 || Hkv < 1 || S < 1 || D < 1) return ATTN_ERR_SHAPE;
   if (Hq % Hkv != 0) return ATTN_ERR_SHAPE;
   if (D != kHeadDim) return ATTN_ERR_UNSUPPORTED;
-  if (S % kBlockM != 0) return ATTN_ERR_UNSUPPORTED;
   // row indices are 32-bit signed in the kernel and in TMA coordinates
   const int64_t q_rows = static_cast<int64_t>(B) * Hq * S;
   if (q_rows >= (int64_t(1) << 31)) return ATTN_ERR_SHAPE;
@@ -176,7 +175,8 @@ bool encode_call_maps(CallMaps* m, const void* q, const void* k, const void* v, 
 // The fused pass over every item, then the hi+lo pass over the items it
 // listed.
 attn_status launch_passes(const CallMaps& m, const FwdParams& p, int dev, cudaStream_t cs) {
-  if (kPairFusedPass) {
+  // the pair kernel takes whole 128-row blocks only
+  if (kPairFusedPass && p.s_tail == kBlockM) {
     const int pairs = p.n_items < g_dev_pairs[dev] ? p.n_items : g_dev_pairs[dev];
     pair::attn_fwd_pair_kernel<<<2 * pairs, pair::kThreads, pair_smem_bytes(), cs>>>(
         m.q, m.k_half, m.v, p);
@@ -207,7 +207,7 @@ const char* attn_status_string(attn_status s) {
     case ATTN_ERR_SHAPE: return "ATTN_ERR_SHAPE: invalid or too large sizes";
     case ATTN_ERR_ALIGN: return "ATTN_ERR_ALIGN: a device pointer is not 16-byte aligned";
     case ATTN_ERR_UNSUPPORTED:
-      return "ATTN_ERR_UNSUPPORTED: needs D == 128, S % 128 == 0 and an sm_100 device";
+      return "ATTN_ERR_UNSUPPORTED: needs D == 128 and an sm_100 device";
     case ATTN_ERR_CUDA: return "ATTN_ERR_CUDA: a CUDA call failed";
     case ATTN_ERR_DEVICE_TIMEOUT: return "ATTN_ERR_DEVICE_TIMEOUT: a kernel wait ran out";
     case ATTN_ERR_WORKSPACE: return "ATTN_ERR_WORKSPACE: device workspace too small";
@@ -245,7 +245,8 @@ attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float
   p.Hkv = Hkv;
   p.S = S;
   p.causal = causal ? 1 : 0;
-  p.n_qb = S / kBlockM;
+  p.n_qb = (S + kBlockM - 1) / kBlockM;
+  p.s_tail = S - (p.n_qb - 1) * kBlockM;
   p.n_qb2 = (p.n_qb + 1) / 2;
   p.group = Hq / Hkv;
   p.n_items = B * Hq * p.n_qb2;
@@ -404,7 +405,7 @@ extern "C" attn_status attn_fwd_noalloc(const void* q, const void* k, const void
   if (st != ATTN_OK) return st;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
     return ATTN_ERR_ALIGN;
-  const int n_qb = S / kBlockM;
+  const int n_qb = (S + kBlockM - 1) / kBlockM;
   const int n_qb2 = (n_qb + 1) / 2;
   const long long n_items = static_cast<long long>(B) * Hq * n_qb2;
   if (n_items > kNoAllocMaxItems) return ATTN_ERR_TOO_LARGE;
@@ -426,6 +427,7 @@ extern "C" attn_status attn_fwd_noalloc(const void* q, const void* k, const void
   p.S = S;
   p.causal = causal ? 1 : 0;
   p.n_qb = n_qb;
+  p.s_tail = S - (n_qb - 1) * kBlockM;
   p.n_qb2 = n_qb2;
   p.group = Hq / Hkv;
   p.n_items = static_cast<int>(n_items);

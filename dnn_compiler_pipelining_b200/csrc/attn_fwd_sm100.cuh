@@ -77,8 +77,8 @@ constexpr int kProducerWarp = 12;   // Q and K
 constexpr int kMmaWarp = 13;
 constexpr int kProducerVWarp = 14;  // V
 constexpr int kRegsSoftmax = 192;
-constexpr int kRegsEpilogue = 64;
-constexpr int kRegsOther = 64;
+constexpr int kRegsEpilogue = 80;
+constexpr int kRegsOther = 48;
 static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsEpilogue + 128 * kRegsOther <= kThreads * 128,
               "register split exceeds the launch allocation");
 
@@ -95,7 +95,8 @@ struct FwdParams {
   int B, Hq, Hkv, S;
   int causal;
   int n_items;       // B * Hq * n_qb2
-  int n_qb;          // S / 128 row blocks
+  int n_qb;          // ceil(S / 128) row (and key) blocks
+  int s_tail;        // rows (keys) in the last block, 1..128
   int n_qb2;         // ceil(n_qb / 2) items per (batch, head)
   int group;         // Hq / Hkv
   float scale_log2;  // log2(e) / sqrt(D)
@@ -460,7 +461,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float l = sm->stat_l[x][r];
           mbar_arrive(smem_addr(&sm->stats_free[x]));  // the softmax may write the next item's
           const float inv_l = 1.0f / l;
-          const int row = (it.b * p.Hq + it.hq) * p.S + it.qb2 * kItemRows + x * kBlockM + r;
+          // rows past S (a ragged last block) are computed but not stored
+          const int i_row = it.qb2 * kItemRows + x * kBlockM + r;
+          const bool valid = i_row < p.S;
+          const int row = (it.b * p.Hq + it.hq) * p.S + i_row;
           uint4* orow = reinterpret_cast<uint4*>(p.o + static_cast<size_t>(row) * kHeadDim);
           float omax = 0.f;
 #pragma unroll
@@ -482,13 +486,13 @@ __global__ void __launch_bounds__(kThreads, 1)
               pk.y = pack_half2(f[2], f[3]);
               pk.z = pack_half2(f[4], f[5]);
               pk.w = pack_half2(f[6], f[7]);
-              orow[c * 2 + v4] = pk;
+              if (valid) orow[c * 2 + v4] = pk;
             }
           }
           tc_fence_before();
           mbar_arrive(smem_addr(&sm->o_free[x]));
-          p.lse[row] = (m_use + log2f(l)) * kLn2;
-          flag |= omax >= kRedoThreshold;
+          if (valid) p.lse[row] = (m_use + log2f(l)) * kLn2;
+          flag |= valid && omax >= kRedoThreshold;
         }
         if (!ok) break;
         if (kMode == 0) {
@@ -530,6 +534,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int n_x = it.n_kv[x];
         if (n_x == 0) continue;
         const int diag = p.causal ? n_x - 1 : -1;
+        const int tail_blk = p.causal ? -1 : n_x - 1;
         float m_use = -INFINITY;
         float l = 0.f;
         bool ok = true;
@@ -548,10 +553,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_wait_ld();
 #pragma unroll
           for (int c = 0; c < 4; ++c) reg_dep32(&u[c * 32]);
-          if (j == diag) {
+          // causal: the diagonal block keeps keys <= row.  Non-causal: a
+          // ragged last block keeps its first s_tail keys (the rows past S
+          // belong to the next head or lie past the tensor, zero-filled);
+          // with the causal mask the diagonal block already hides them.
+          if (j == diag || (j == tail_blk && p.s_tail < kBlockN)) {
+            const int lim = j == diag ? r : p.s_tail - 1;
 #pragma unroll
             for (int c = 0; c < 128; ++c)
-              if (c > r) u[c] = 0xff800000u;  // -inf
+              if (c > lim) u[c] = 0xff800000u;  // -inf
           }
           // row max: 8 independent chains (chain t takes columns t, t + 8,
           // ..., t + 120) of 3-input max, then a tree

@@ -42,6 +42,44 @@ def test_small_stress_full(B, Hq, Hkv, S, causal):
     parity.full_check(B, Hq, Hkv, S, 128, causal, seed=11, qk_std=4.0)
 
 
+# S not a multiple of 128: the last row / key block is ragged
+RAGGED = [(1, 4, 2, 1), (1, 4, 2, 77), (2, 4, 2, 200), (1, 8, 2, 383), (2, 6, 3, 1000)]
+
+
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("B,Hq,Hkv,S", RAGGED)
+def test_ragged_full(B, Hq, Hkv, S, causal):
+    """Keys past S are masked and rows past S are computed but not stored."""
+    parity.full_check(B, Hq, Hkv, S, 128, causal, seed=13)
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_ragged_stress_full(causal):
+    parity.full_check(1, 8, 2, 329, 128, causal, seed=17, qk_std=4.0)
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_ragged_writes_stay_in_bounds(causal):
+    """O and LSE end inside larger buffers whose tails hold a sentinel: the
+    last head's rows past S (inside the ragged block) must not be stored."""
+    B, Hq, Hkv, S, D = 1, 2, 1, 150, 128
+    q, k, v = make_qkv(B, Hq, Hkv, S, D, seed=19, device="cuda")
+    n_o, n_l, pad = B * Hq * S * D, B * Hq * S, 128 * D
+    o_buf = torch.full((n_o + pad,), 7.0, dtype=torch.float16, device="cuda")
+    l_buf = torch.full((n_l + 4 * 128,), 7.0, dtype=torch.float32, device="cuda")
+    o = o_buf[:n_o].view(B, Hq, S, D)
+    lse = l_buf[:n_l].view(B, Hq, S)
+    attn.attn_fwd(q, k, v, causal, o=o, lse=lse)
+    st, site = attn.device_status()
+    assert st == attn.ATTN_OK, "device status %d at site %#x" % (st, site)
+    assert bool((o_buf[n_o:] == 7.0).all().item()), "O written past its end"
+    assert bool((l_buf[n_l:] == 7.0).all().item()), "LSE written past its end"
+    o_ref, lse_ref = parity.oracle.attention(q.cpu().double().numpy(), k.cpu().double().numpy(),
+                                             v.cpu().double().numpy(), causal)
+    parity.assert_close(o.cpu().double().numpy(), o_ref, lse.cpu().double().numpy(), lse_ref,
+                        "ragged in-bounds causal=%d" % causal)
+
+
 def test_llama3_8b_s512_b1_full():
     w = WORKLOADS["llama3-8b-s512-b1"]
     parity.full_check(w["B"], w["Hq"], w["Hkv"], w["S"], w["D"], w["causal"], seed=0)
