@@ -77,7 +77,10 @@ unsigned int* redo_list(int dev, cudaStream_t stream) {
 // (793 vs 1003 TFLOP/s at B=64, S=8192, causal).
 constexpr bool kPairFusedPass = false;
 
-size_t fwd_smem_bytes() { return sizeof(SharedFwd); }  // the kernel checks 1 KiB alignment
+// the kernel checks 1 KiB alignment of the dynamic shared memory base
+size_t fwd_smem_bytes(int D = kHeadDim) {
+  return D == 64 ? sizeof(SharedFwdT<64>) : sizeof(SharedFwdT<128>);
+}
 size_t pair_smem_bytes() { return sizeof(pair::SharedPair); }
 
 attn_status device_setup(int* dev_out) {
@@ -102,10 +105,14 @@ attn_status device_setup(int* dev_out) {
     if (cudaDeviceGetAttribute(&g_dev_sms[dev], cudaDevAttrMultiProcessorCount, dev) !=
         cudaSuccess)
       return ATTN_ERR_CUDA;
-    if (cudaFuncSetAttribute(attn_fwd_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(fwd_smem_bytes())) != cudaSuccess ||
-        cudaFuncSetAttribute(attn_fwd_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(fwd_smem_bytes())) != cudaSuccess ||
+    if (cudaFuncSetAttribute(attn_fwd_kernel<0, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(fwd_smem_bytes(128))) != cudaSuccess ||
+        cudaFuncSetAttribute(attn_fwd_kernel<1, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(fwd_smem_bytes(128))) != cudaSuccess ||
+        cudaFuncSetAttribute(attn_fwd_kernel<0, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(fwd_smem_bytes(64))) != cudaSuccess ||
+        cudaFuncSetAttribute(attn_fwd_kernel<1, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(fwd_smem_bytes(64))) != cudaSuccess ||
         cudaFuncSetAttribute(pair::attn_fwd_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(pair_smem_bytes())) != cudaSuccess)
       return ATTN_ERR_CUDA;
@@ -127,14 +134,14 @@ attn_status device_setup(int* dev_out) {
   return g_dev_state[dev].load() == 1 ? ATTN_OK : ATTN_ERR_UNSUPPORTED;
 }
 
-// 2-D view [rows, 128] fp16 of a dense [.., S, 128] tensor; 64 x 128 boxes
-// (one 128-byte swizzle panel of 128 rows).
-bool encode_rows_map(CUtensorMap* map, const void* base, uint64_t rows,
+// 2-D view [rows, D] fp16 of a dense [.., S, D] tensor; 64 x box_rows boxes
+// (one 128-byte swizzle panel).
+bool encode_rows_map(CUtensorMap* map, const void* base, uint64_t rows, int D,
                      uint32_t box_rows = kBlockM) {
   auto fn = encode_fn();
   if (!fn) return false;
-  cuuint64_t dims[2] = {static_cast<cuuint64_t>(kHeadDim), static_cast<cuuint64_t>(rows)};
-  cuuint64_t strides[1] = {static_cast<cuuint64_t>(kHeadDim) * 2};
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(D) * 2};
   cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides,
@@ -148,7 +155,7 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 attn_status validate_sizes(int B, int Hq, int Hkv, int S, int D) {
   if (B < 1 || Hq < 1 || Hkv < 1 || S < 1 || D < 1) return ATTN_ERR_SHAPE;
   if (Hq % Hkv != 0) return ATTN_ERR_SHAPE;
-  if (D != kHeadDim) return ATTN_ERR_UNSUPPORTED;
+  if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
   // row indices are 32-bit signed in the kernel and in TMA coordinates
   const int64_t q_rows = static_cast<int64_t>(B) * Hq * S;
   if (q_rows >= (int64_t(1) << 31)) return ATTN_ERR_SHAPE;
@@ -165,30 +172,37 @@ struct CallMaps {
 };
 
 bool encode_call_maps(CallMaps* m, const void* q, const void* k, const void* v, int B, int Hq,
-                      int Hkv, int S) {
+                      int Hkv, int S, int D) {
   const uint64_t q_rows = static_cast<uint64_t>(B) * Hq * S;
   const uint64_t kv_rows = static_cast<uint64_t>(B) * Hkv * S;
-  return encode_rows_map(&m->q, q, q_rows) && encode_rows_map(&m->k, k, kv_rows) &&
-         encode_rows_map(&m->k_half, k, kv_rows, kBlockM / 2) && encode_rows_map(&m->v, v, kv_rows);
+  return encode_rows_map(&m->q, q, q_rows, D) && encode_rows_map(&m->k, k, kv_rows, D) &&
+         encode_rows_map(&m->k_half, k, kv_rows, D, kBlockM / 2) &&
+         encode_rows_map(&m->v, v, kv_rows, D);
 }
 
 // The fused pass over every item, then the hi+lo pass over the items it
 // listed.
-attn_status launch_passes(const CallMaps& m, const FwdParams& p, int dev, cudaStream_t cs) {
-  // the pair kernel takes whole 128-row blocks only
-  if (kPairFusedPass && p.s_tail == kBlockM) {
+template <int kD>
+attn_status launch_passes_d(const CallMaps& m, const FwdParams& p, int dev, cudaStream_t cs) {
+  const int sms = g_dev_sms[dev];
+  // the pair kernel takes D = 128 and whole 128-row blocks only
+  if (kPairFusedPass && kD == 128 && p.s_tail == kBlockM) {
     const int pairs = p.n_items < g_dev_pairs[dev] ? p.n_items : g_dev_pairs[dev];
     pair::attn_fwd_pair_kernel<<<2 * pairs, pair::kThreads, pair_smem_bytes(), cs>>>(
         m.q, m.k_half, m.v, p);
   } else {
-    const int sms = g_dev_sms[dev];
-    attn_fwd_kernel<0><<<p.n_items < sms ? p.n_items : sms, kThreads, fwd_smem_bytes(), cs>>>(
-        m.q, m.k, m.v, p);
+    attn_fwd_kernel<0, kD><<<p.n_items < sms ? p.n_items : sms, kThreads, fwd_smem_bytes(kD),
+                             cs>>>(m.q, m.k, m.v, p);
   }
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
-  attn_fwd_kernel<1><<<g_dev_sms[dev], kThreads, fwd_smem_bytes(), cs>>>(m.q, m.k, m.v, p);
+  attn_fwd_kernel<1, kD><<<sms, kThreads, fwd_smem_bytes(kD), cs>>>(m.q, m.k, m.v, p);
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
   return ATTN_OK;
+}
+
+attn_status launch_passes(const CallMaps& m, const FwdParams& p, int D, int dev,
+                          cudaStream_t cs) {
+  return D == 64 ? launch_passes_d<64>(m, p, dev, cs) : launch_passes_d<128>(m, p, dev, cs);
 }
 
 }  // namespace
@@ -207,7 +221,7 @@ const char* attn_status_string(attn_status s) {
     case ATTN_ERR_SHAPE: return "ATTN_ERR_SHAPE: invalid or too large sizes";
     case ATTN_ERR_ALIGN: return "ATTN_ERR_ALIGN: a device pointer is not 16-byte aligned";
     case ATTN_ERR_UNSUPPORTED:
-      return "ATTN_ERR_UNSUPPORTED: needs D == 128 and an sm_100 device";
+      return "ATTN_ERR_UNSUPPORTED: needs D == 64 or 128 and an sm_100 device";
     case ATTN_ERR_CUDA: return "ATTN_ERR_CUDA: a CUDA call failed";
     case ATTN_ERR_DEVICE_TIMEOUT: return "ATTN_ERR_DEVICE_TIMEOUT: a kernel wait ran out";
     case ATTN_ERR_WORKSPACE: return "ATTN_ERR_WORKSPACE: device workspace too small";
@@ -235,7 +249,7 @@ attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float
   if (st != ATTN_OK) return st;
 
   CallMaps maps;
-  if (!encode_call_maps(&maps, q, k, v, B, Hq, Hkv, S)) return ATTN_ERR_CUDA;
+  if (!encode_call_maps(&maps, q, k, v, B, Hq, Hkv, S, D)) return ATTN_ERR_CUDA;
 
   FwdParams p;
   p.o = static_cast<__half*>(o);
@@ -257,7 +271,7 @@ attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float
   if (!p.redo) return ATTN_ERR_CUDA;
   p.redo_capacity = kRedoCapacity;
 
-  return launch_passes(maps, p, dev, cs);
+  return launch_passes(maps, p, D, dev, cs);
 }
 
 size_t attn_fwd_host_workspace_bytes(int B, int Hq, int Hkv, int S, int D) {
@@ -416,7 +430,7 @@ extern "C" attn_status attn_fwd_noalloc(const void* q, const void* k, const void
   if (!scratch) return ATTN_ERR_CUDA;
 
   CallMaps maps;
-  if (!encode_call_maps(&maps, q, k, v, B, Hq, Hkv, S)) return ATTN_ERR_CUDA;
+  if (!encode_call_maps(&maps, q, k, v, B, Hq, Hkv, S, D)) return ATTN_ERR_CUDA;
 
   FwdParams p;
   p.o = static_cast<__half*>(o);
@@ -440,5 +454,5 @@ extern "C" attn_status attn_fwd_noalloc(const void* q, const void* k, const void
   // the shared array keeps the previous call's header: start from an empty list
   if (cudaMemsetAsync(scratch, 0, kRedoHeaderWords * sizeof(unsigned int), cs) != cudaSuccess)
     return ATTN_ERR_CUDA;
-  return launch_passes(maps, p, dev, cs);
+  return launch_passes(maps, p, D, dev, cs);
 }

@@ -121,13 +121,21 @@ enum WaitSite : uint32_t {
   kSiteDrain = 0x501,
 };
 
-// Shared memory: 224 KiB of tiles first (each 1 KiB aligned, as the 128-byte
-// swizzle needs), then the row statistics and the barriers.  The dynamic
-// shared memory base is checked to be 1 KiB aligned at launch.
-struct SharedFwd {
-  uint8_t q[2][kTileBytes];
-  uint8_t k[kStagesK][kTileBytes];
-  uint8_t v[kStagesV][kTileBytes];
+// Bytes of one 128-row fp16 tile of head dimension kD (kD / 64 panels of 64
+// columns, 128 bytes per row of a panel).
+template <int kD>
+__host__ __device__ constexpr uint32_t tile_bytes() {
+  return static_cast<uint32_t>(kBlockM) * kD * 2;
+}
+
+// Shared memory: the tiles first (224 KiB at kD = 128; each 1 KiB aligned,
+// as the 128-byte swizzle needs), then the row statistics and the barriers.
+// The dynamic shared memory base is checked to be 1 KiB aligned at launch.
+template <int kD>
+struct SharedFwdT {
+  uint8_t q[2][tile_bytes<kD>()];
+  uint8_t k[kStagesK][tile_bytes<kD>()];
+  uint8_t v[kStagesV][tile_bytes<kD>()];
   float stat_m[2][kBlockM];  // [tile][row], handed from softmax to epilogue
   float stat_l[2][kBlockM];
   uint64_t q_full, q_empty;
@@ -141,7 +149,8 @@ struct SharedFwd {
   unsigned int n_listed;
 };
 
-static_assert(sizeof(SharedFwd) <= 232448, "shared memory exceeds the 227 KiB per-block limit");
+static_assert(sizeof(SharedFwdT<128>) <= 232448, "shared memory exceeds the 227 KiB per-block limit");
+using SharedFwd = SharedFwdT<128>;
 
 struct Item {
   int b, hq, g, qb2;
@@ -196,9 +205,9 @@ __device__ __forceinline__ uint32_t ring_parity(int rc) {
   return (rc / kDepth) & 1;
 }
 
-// S_X(j) = Q_X K^T: 8 MMAs of K = 16 over the head dimension.  Both operands
-// are K-major; 16 columns are 32 bytes inside a 128-byte swizzled row and
-// columns 64..127 live in the second panel.
+// S_X(j) = Q_X K^T: kD / 16 MMAs of K = 16 over the head dimension.  Both
+// operands are K-major; 16 columns are 32 bytes inside a 128-byte swizzled
+// row and columns 64..127 (kD = 128) live in the second panel.
 // A descriptor's start address sits in its low bits (16-byte units), so a
 // descriptor for base + off is the base descriptor plus off >> 4 (shared
 // memory offsets stay below 256 KiB, so no carry leaves the field).
@@ -208,7 +217,9 @@ __device__ __forceinline__ void qk_step(uint32_t d_tmem, uint64_t qd, uint64_t k
   mma_f16_ss_off<off, off>(d_tmem, qd, kd, idesc, kk > 0 ? 1u : 0u);
 }
 
+template <int kD>
 __device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_s, uint32_t k_s) {
+  static_assert(kD == 64 || kD == 128, "head dimension 64 or 128");
   const uint32_t idesc = idesc_f16_f32(kBlockM, kBlockN, false, false);
   const uint64_t qd = smem_desc_sw128(q_s, 16, 1024);
   const uint64_t kd = smem_desc_sw128(k_s, 16, 1024);
@@ -216,15 +227,17 @@ __device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_s, uint32_t
   qk_step<1>(d_tmem, qd, kd, idesc);
   qk_step<2>(d_tmem, qd, kd, idesc);
   qk_step<3>(d_tmem, qd, kd, idesc);
-  qk_step<4>(d_tmem, qd, kd, idesc);
-  qk_step<5>(d_tmem, qd, kd, idesc);
-  qk_step<6>(d_tmem, qd, kd, idesc);
-  qk_step<7>(d_tmem, qd, kd, idesc);
+  if constexpr (kD == 128) {
+    qk_step<4>(d_tmem, qd, kd, idesc);
+    qk_step<5>(d_tmem, qd, kd, idesc);
+    qk_step<6>(d_tmem, qd, kd, idesc);
+    qk_step<7>(d_tmem, qd, kd, idesc);
+  }
 }
 
 // O_X (+)= P V: A = P from TMEM (8 columns = 16 keys per MMA), B = V, an
-// MN-major operand (16 keys = two 8-row groups of 1 KiB; the two 64-column
-// halves of D are a panel apart).
+// MN-major operand of N = kD (16 keys = two 8-row groups of 1 KiB; at kD = 128
+// the two 64-column halves of D are a panel apart).
 template <int kk>
 __device__ __forceinline__ void pv_step(uint32_t o_tmem, uint32_t p_tmem, uint64_t vd,
                                         uint32_t idesc, uint32_t acc) {
@@ -233,9 +246,10 @@ __device__ __forceinline__ void pv_step(uint32_t o_tmem, uint32_t p_tmem, uint64
   mma_f16_ts_off<a_off, b_off>(o_tmem, p_tmem, vd, idesc, (acc || kk > 0) ? 1u : 0u);
 }
 
+template <int kD>
 __device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint32_t v_s,
                                          bool accumulate) {
-  const uint32_t idesc = idesc_f16_f32(kBlockM, kHeadDim, false, true);
+  const uint32_t idesc = idesc_f16_f32(kBlockM, kD, false, true);
   const uint64_t vd = smem_desc_sw128(v_s, kPanelBytes, 1024);
   const uint32_t acc = accumulate ? 1u : 0u;
   pv_step<0>(o_tmem, p_tmem, vd, idesc, acc);
@@ -249,13 +263,15 @@ __device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint3
 }
 
 // kMode 0: the fused pass over every item; kMode 1: the redo pass over the
-// listed items with hi + lo probabilities.
-template <int kMode>
+// listed items with hi + lo probabilities.  kD: the head dimension, 64 or 128.
+template <int kMode, int kD = 128>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+  constexpr uint32_t kTile = tile_bytes<kD>();
+  constexpr int kPanels = kD / 64;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  SharedFwd* sm = reinterpret_cast<SharedFwd*>(smem_raw);
+  SharedFwdT<kD>* sm = reinterpret_cast<SharedFwdT<kD>*>(smem_raw);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const uint64_t to = p.timeout_ns;
@@ -333,12 +349,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             const int q_row = (it.b * p.Hq + it.hq) * p.S + it.qb2 * kItemRows;
             const uint32_t qf = smem_addr(&sm->q_full);
-            mbar_arrive_expect_tx(qf, 2 * kTileBytes);
+            mbar_arrive_expect_tx(qf, 2 * kTile);
 #pragma unroll
             for (int x = 0; x < 2; ++x) {
               const uint32_t q_s = smem_addr(sm->q[x]);
-              tma_load_2d_hint(q_s, &tm_q, qf, 0, q_row + x * kBlockM, once);
-              tma_load_2d_hint(q_s + kPanelBytes, &tm_q, qf, 64, q_row + x * kBlockM, once);
+#pragma unroll
+              for (int pn = 0; pn < kPanels; ++pn)
+                tma_load_2d_hint(q_s + pn * kPanelBytes, &tm_q, qf, 64 * pn, q_row + x * kBlockM,
+                                 once);
             }
           }
           const int kv_row = (it.b * p.Hkv + it.g) * p.S;
@@ -354,9 +372,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t full = smem_addr(is_v ? &sm->v_full[st] : &sm->k_full[st]);
             const uint32_t dst = smem_addr(is_v ? sm->v[st] : sm->k[st]);
             const CUtensorMap* map = is_v ? &tm_v : &tm_k;
-            mbar_arrive_expect_tx(full, kTileBytes);
-            tma_load_2d_hint(dst, map, full, 0, kv_row + j * kBlockN, keep);
-            tma_load_2d_hint(dst + kPanelBytes, map, full, 64, kv_row + j * kBlockN, keep);
+            mbar_arrive_expect_tx(full, kTile);
+#pragma unroll
+            for (int pn = 0; pn < kPanels; ++pn)
+              tma_load_2d_hint(dst + pn * kPanelBytes, map, full, 64 * pn, kv_row + j * kBlockN,
+                               keep);
           }
         }
         if (*abort) {
@@ -406,8 +426,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ++pcnt[x];
                 tc_fence_after();
                 const uint32_t v_s = smem_addr(sm->v[st_v]);
-                issue_pv(tmem + tmem_o_col(x), tmem + tmem_s_col(x), v_s, j - 1 > 0);
-                if (hilo) issue_pv(tmem + tmem_o_col(x), tmem + tmem_s_col(x) + 64, v_s, true);
+                issue_pv<kD>(tmem + tmem_o_col(x), tmem + tmem_s_col(x), v_s, j - 1 > 0);
+                if (hilo) issue_pv<kD>(tmem + tmem_o_col(x), tmem + tmem_s_col(x) + 64, v_s, true);
                 if (j == n_x) tc_commit(smem_addr(&sm->o_done[x]));
               }
               if (j < n_x) {
@@ -418,7 +438,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                   if (!ok) break;
                   tc_fence_after();
                 }
-                issue_qk(tmem + tmem_s_col(x), smem_addr(sm->q[x]), smem_addr(sm->k[st_k]));
+                issue_qk<kD>(tmem + tmem_s_col(x), smem_addr(sm->q[x]), smem_addr(sm->k[st_k]));
                 tc_commit(smem_addr(&sm->s_full[x]));
               }
             }
@@ -465,10 +485,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int i_row = it.qb2 * kItemRows + x * kBlockM + r;
           const bool valid = i_row < p.S;
           const int row = (it.b * p.Hq + it.hq) * p.S + i_row;
-          uint4* orow = reinterpret_cast<uint4*>(p.o + static_cast<size_t>(row) * kHeadDim);
+          uint4* orow = reinterpret_cast<uint4*>(p.o + static_cast<size_t>(row) * kD);
           float omax = 0.f;
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {
+          for (int c = 0; c < kD / 16; ++c) {
             uint32_t w[16];
             tmem_ld16(lane_base + tmem_o_col(x) + c * 16, w);
             tmem_wait_ld();
@@ -587,7 +607,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               // O_X holds P(j-1) V_{j-1} already (it completed before S(j))
               const float alpha = grow ? ex2_approx(m_use - cand) : 1.0f;
 #pragma unroll 1
-              for (int c = 0; c < 4; ++c) {
+              for (int c = 0; c < kD / 32; ++c) {
                 uint32_t w[32];
                 tmem_ld32(o_t + c * 32, w);
                 tmem_wait_ld();

@@ -54,7 +54,7 @@ typedef enum attn_status {
   ATTN_ERR_NULL = 1,           /* a required pointer is NULL */
   ATTN_ERR_SHAPE = 2,          /* B,Hq,Hkv,S < 1, Hq % Hkv != 0, or a size overflows */
   ATTN_ERR_ALIGN = 3,          /* a device pointer is not 16-byte aligned */
-  ATTN_ERR_UNSUPPORTED = 4,    /* D != 128, or not an sm_100 device */
+  ATTN_ERR_UNSUPPORTED = 4,    /* D not 64 or 128, or not an sm_100 device */
   ATTN_ERR_CUDA = 5,           /* a CUDA runtime / driver call failed */
   ATTN_ERR_DEVICE_TIMEOUT = 6, /* a kernel wait ran out; results are invalid */
   ATTN_ERR_WORKSPACE = 7,      /* the device workspace given is too small */
@@ -67,8 +67,9 @@ typedef enum attn_status {
  *   k, v: device, fp16 [B, Hkv, S, D], 16-byte aligned, read only.
  *   o   : device, fp16 [B, Hq, S, D], 16-byte aligned, written.
  *   lse : device, fp32 [B, Hq, S], 16-byte aligned, written (must not be NULL).
- *   B, Hq, Hkv, S, D: sizes; Hq % Hkv == 0; D == 128; any S >= 1 (a last
- *   block of fewer than 128 rows is computed with the keys past S masked).
+ *   B, Hq, Hkv, S, D: sizes; Hq % Hkv == 0; D == 64 or 128; any S >= 1 (a
+ *   last block of fewer than 128 rows is computed with the keys past S
+ *   masked).
  *   causal: nonzero for the causal mask j <= i (square, Sq == Sk == S).
  *   stream: cudaStream_t to launch on.
  * Returns ATTN_OK once the kernels are enqueued; errors as listed above.  The

@@ -57,7 +57,8 @@ def test_validation_before_launch(lib):
     assert call(lib, B=0) == SHAPE
     assert call(lib, Hkv=3) == SHAPE          # Hq % Hkv != 0
     assert call(lib, Hq=0) == SHAPE
-    assert call(lib, D=64) == UNSUP
+    assert call(lib, D=96) == UNSUP
+    assert call(lib, D=256) == UNSUP
     assert call(lib, B=65536, Hq=1, Hkv=1, S=128) == SHAPE
     assert call(lib, B=64, Hq=64, Hkv=8, S=1 << 20) == SHAPE  # row index overflow
     assert call(lib, q=FAKE + 8) == ALIGN

@@ -80,6 +80,28 @@ def test_ragged_writes_stay_in_bounds(causal):
                         "ragged in-bounds causal=%d" % causal)
 
 
+# head dimension 64: one 64-column panel per tile, 4 K-steps in Q K^T, N = 64 in P V
+D64 = [(1, 4, 2, 128), (2, 8, 2, 384), (1, 6, 3, 200), (1, 4, 1, 1000)]
+
+
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("B,Hq,Hkv,S", D64)
+def test_d64_full(B, Hq, Hkv, S, causal):
+    parity.full_check(B, Hq, Hkv, S, 64, causal, seed=23)
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_d64_stress_full(causal):
+    parity.full_check(1, 8, 2, 512, 64, causal, seed=29, qk_std=4.0)
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_d64_sampled(causal):
+    q, k, v = make_qkv(4, 32, 8, 4096, 64, seed=31, device="cuda")
+    o, lse = parity.run_gpu(q, k, v, causal)
+    parity.sampled_check(q, k, v, o, lse, causal, n_random=512, seed=31)
+
+
 def test_llama3_8b_s512_b1_full():
     w = WORKLOADS["llama3-8b-s512-b1"]
     parity.full_check(w["B"], w["Hq"], w["Hkv"], w["S"], w["D"], w["causal"], seed=0)
@@ -171,7 +193,7 @@ def test_bounded_wait_reports_timeout():
 
 
 def test_unsupported_shape_raises():
-    q = torch.zeros(1, 2, 128, 64, dtype=torch.float16, device="cuda")
+    q = torch.zeros(1, 2, 128, 96, dtype=torch.float16, device="cuda")
     with pytest.raises(attn.AttnError):
         attn.attn_fwd(q, q, q)
 
