@@ -50,6 +50,11 @@ def _load():
                                              _f64p, _f64p]
         lib.oracle_attn_probs_row_f64.argtypes = [_f64p, _f64p, ctypes.c_int64, ctypes.c_int64,
                                                   ctypes.c_int64, ctypes.c_int, _f64p, _f64p]
+        lib.oracle_attn_fwd_qk_f64.argtypes = [_f64p, _f64p, _f64p, _f64p, _f64p] + \
+            [ctypes.c_int64] * 6 + [ctypes.c_int]
+        lib.oracle_attn_rows_qk_f64.argtypes = [_f64p, _i64p, ctypes.c_int64, _f64p, _f64p,
+                                                ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+                                                ctypes.c_int, _f64p, _f64p]
         lib.oracle_num_threads.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -106,6 +111,40 @@ def probs_row(q_vec, k_head, i: int, causal: bool):
     if rc != 0:
         raise ValueError("oracle_attn_probs_row_f64 failed (%d)" % rc)
     return p, lse.value
+
+
+def attention_qk(q, k, v, causal: bool):
+    """Sq query rows over Sk keys.  q: [B,Hq,Sq,D]; k, v: [B,Hkv,Sk,D].  The causal
+    window is aligned at the bottom right (query i sees keys j <= i + Sk - Sq).
+    Returns (O [B,Hq,Sq,D], LSE [B,Hq,Sq]) in fp64."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, Hq, Sq, D = q.shape
+    Hkv, Sk = k.shape[1], k.shape[2]
+    if k.shape != (B, Hkv, Sk, D) or v.shape != k.shape:
+        raise ValueError("shape mismatch: q %s k %s v %s" % (q.shape, k.shape, v.shape))
+    o = np.empty_like(q)
+    lse = np.empty((B, Hq, Sq), dtype=np.float64)
+    rc = _load().oracle_attn_fwd_qk_f64(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
+                                        B, Hq, Hkv, Sq, Sk, D, int(bool(causal)))
+    if rc != 0:
+        raise ValueError("oracle_attn_fwd_qk_f64 failed (%d)" % rc)
+    return o, lse
+
+
+def attention_rows_qk(q_rows, pos, k_head, v_head, Sq: int, causal: bool):
+    """Selected query rows (positions in [0, Sq)) of one head over Sk keys."""
+    q_rows, k_head, v_head = _f64(q_rows), _f64(k_head), _f64(v_head)
+    pos = np.ascontiguousarray(np.asarray(pos, dtype=np.int64))
+    n, D = q_rows.shape
+    Sk = k_head.shape[0]
+    o = np.empty((n, D), dtype=np.float64)
+    lse = np.empty((n,), dtype=np.float64)
+    rc = _load().oracle_attn_rows_qk_f64(_ptr(q_rows), _ptr(pos, _i64p), n, _ptr(k_head),
+                                         _ptr(v_head), int(Sq), Sk, D, int(bool(causal)),
+                                         _ptr(o), _ptr(lse))
+    if rc != 0:
+        raise ValueError("oracle_attn_rows_qk_f64 failed (%d)" % rc)
+    return o, lse
 
 
 def num_threads() -> int:

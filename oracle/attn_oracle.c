@@ -25,7 +25,8 @@
  *                                  scaled logits)
  *
  * Layout: Q, O are [B, Hq, S, D]; K, V are [B, Hkv, S, D]; LSE is [B, Hq, S];
- * all dense, row-major, fp64.  Every function returns 0 on success and a
+ * all dense, row-major, fp64.  The *_qk_* functions at the end take Sq query
+ * rows over Sk keys, with the causal window aligned at the bottom right.  Every function returns 0 on success and a
  * negative value on a bad argument; it never aborts.
  */
 #include <math.h>
@@ -147,6 +148,124 @@ int oracle_attn_fwd_f64(const double* q, const double* k, const double* v,
             const int64_t row = (b * Hq + hq) * S + i;
             if (oracle_attn_row_f64(q + row * D, kh, vh, i, S, D, causal,
                                     o + row * D, lse + row, scratch)) {
+#pragma omp atomic write
+              bad = 1;
+            }
+          }
+      free(scratch);
+    }
+  }
+  return bad ? -3 : 0;
+}
+
+/*
+ * Different query and key lengths: Sq query rows over Sk keys.  The causal
+ * window is aligned at the bottom right -- query i sees keys
+ * j <= i + (Sk - Sq) -- so the last query sees every key, and Sq == Sk is the
+ * square case above.  A causal query with no visible key (Sq > Sk and
+ * i < Sq - Sk) is rejected (-4): softmax over an empty set is undefined.
+ * Layout: Q, O [B, Hq, Sq, D]; K, V [B, Hkv, Sk, D]; LSE [B, Hq, Sq].
+ */
+static int64_t qk_visible_keys(int64_t i, int64_t Sq, int64_t Sk, int causal) {
+  if (!causal) return Sk;
+  const int64_t last = i + (Sk - Sq); /* the last visible key */
+  return last + 1 < Sk ? last + 1 : Sk;
+}
+
+/*
+ * One query row i of a head: o[D] and its LSE.  k, v: [Sk, D] of the kv
+ * head; scratch: caller-provided [Sk] doubles.
+ */
+int oracle_attn_row_qk_f64(const double* q, const double* k, const double* v,
+                           int64_t i, int64_t Sq, int64_t Sk, int64_t D,
+                           int causal, double* o, double* lse,
+                           double* scratch) {
+  if (!q || !k || !v || !o || !lse || !scratch) return -1;
+  if (D <= 0 || Sq <= 0 || Sk <= 0 || i < 0 || i >= Sq) return -1;
+  const int64_t nk = qk_visible_keys(i, Sq, Sk, causal);
+  if (nk < 1) return -4;
+  const double scale = pow((double)D, -0.5);
+  /* pass 1: the scaled logits of the visible keys, and their maximum */
+  double mx = -INFINITY;
+  for (int64_t j = 0; j < nk; ++j) {
+    double acc = 0.0;
+    for (int64_t d = 0; d < D; ++d) acc += q[d] * k[D * j + d];
+    scratch[j] = acc * scale;
+    if (scratch[j] > mx) mx = scratch[j];
+  }
+  /* pass 2: weights exp(s - max), their sum, and the weighted values */
+  double sum = 0.0;
+  for (int64_t j = 0; j < nk; ++j) {
+    scratch[j] = exp(scratch[j] - mx);
+    sum += scratch[j];
+  }
+  for (int64_t d = 0; d < D; ++d) o[d] = 0.0;
+  for (int64_t j = 0; j < nk; ++j)
+    for (int64_t d = 0; d < D; ++d) o[d] += scratch[j] * v[D * j + d];
+  for (int64_t d = 0; d < D; ++d) o[d] /= sum;
+  *lse = mx + log(sum);
+  return 0;
+}
+
+/* Selected rows of one head (positions pos[n] in [0, Sq)). */
+int oracle_attn_rows_qk_f64(const double* q_rows, const int64_t* pos, int64_t n,
+                            const double* k, const double* v, int64_t Sq,
+                            int64_t Sk, int64_t D, int causal, double* o,
+                            double* lse) {
+  if (!q_rows || !pos || !k || !v || !o || !lse || n < 0 || Sq <= 0 || Sk <= 0 ||
+      D <= 0)
+    return -1;
+  for (int64_t r = 0; r < n; ++r)
+    if (pos[r] < 0 || pos[r] >= Sq) return -2;
+  int bad = 0;
+#pragma omp parallel
+  {
+    double* scratch = (double*)malloc(sizeof(double) * (size_t)Sk);
+    if (!scratch) {
+#pragma omp atomic write
+      bad = 1;
+    } else {
+#pragma omp for schedule(dynamic, 4)
+      for (int64_t r = 0; r < n; ++r) {
+        const int rc = oracle_attn_row_qk_f64(q_rows + r * D, k, v, pos[r], Sq, Sk, D,
+                                              causal, o + r * D, lse + r, scratch);
+        if (rc) {
+#pragma omp atomic write
+          bad = rc;
+        }
+      }
+      free(scratch);
+    }
+  }
+  return bad ? (bad < 0 ? bad : -3) : 0;
+}
+
+/* Whole tensors, every (b, hq, i); kv head g = hq / (Hq / Hkv). */
+int oracle_attn_fwd_qk_f64(const double* q, const double* k, const double* v,
+                           double* o, double* lse, int64_t B, int64_t Hq,
+                           int64_t Hkv, int64_t Sq, int64_t Sk, int64_t D,
+                           int causal) {
+  if (!q || !k || !v || !o || !lse) return -1;
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Sq <= 0 || Sk <= 0 || D <= 0) return -1;
+  if (Hq % Hkv != 0) return -2;
+  if (causal && Sq > Sk) return -4;
+  const int64_t heads_per_kv = Hq / Hkv;
+  int bad = 0;
+#pragma omp parallel
+  {
+    double* scratch = (double*)malloc(sizeof(double) * (size_t)Sk);
+    if (!scratch) {
+#pragma omp atomic write
+      bad = 1;
+    } else {
+#pragma omp for collapse(3) schedule(dynamic, 16)
+      for (int64_t b = 0; b < B; ++b)
+        for (int64_t hq = 0; hq < Hq; ++hq)
+          for (int64_t i = 0; i < Sq; ++i) {
+            const int64_t kvh = b * Hkv + hq / heads_per_kv;
+            const int64_t row = (b * Hq + hq) * Sq + i;
+            if (oracle_attn_row_qk_f64(q + row * D, k + kvh * Sk * D, v + kvh * Sk * D, i, Sq,
+                                       Sk, D, causal, o + row * D, lse + row, scratch)) {
 #pragma omp atomic write
               bad = 1;
             }

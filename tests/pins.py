@@ -209,6 +209,70 @@ def check_rows_api(orc):
         assert np.array_equal(o2, o[0, hq, pos]) and np.array_equal(l2, lse[0, hq, pos])
 
 
+def check_qk_suffix(orc):
+    """Bottom-right alignment: causal attention of the last Sq queries over all
+    Sk keys equals the last Sq rows of the square causal problem (whose
+    definition the pins above fix)."""
+    r = _rng(11)
+    B, Hq, Hkv, Sk, D = 1, 4, 2, 37, 16
+    q = r.normal(size=(B, Hq, Sk, D)) * 2
+    k = r.normal(size=(B, Hkv, Sk, D)) * 2
+    v = r.normal(size=(B, Hkv, Sk, D))
+    o_sq, l_sq = orc.attention(q, k, v, True)
+    for sq in (1, 11, 36, 37):
+        o, lse = orc.attention_qk(q[:, :, Sk - sq:], k, v, True)
+        assert np.allclose(o, o_sq[:, :, Sk - sq:], rtol=0, atol=1e-12)
+        assert np.allclose(lse, l_sq[:, :, Sk - sq:], rtol=0, atol=1e-12)
+
+
+def check_qk_library(orc):
+    """Sq != Sk against fp64 torch scaled_dot_product_attention: non-causal, and
+    causal with the bottom-right boolean mask written out (j <= i + Sk - Sq)."""
+    import torch
+    r = _rng(12)
+    B, Hq, Hkv, Sq, Sk, D = 2, 4, 2, 13, 29, 8
+    q = r.normal(size=(B, Hq, Sq, D)) * 2
+    k = r.normal(size=(B, Hkv, Sk, D)) * 2
+    v = r.normal(size=(B, Hkv, Sk, D))
+    tq = torch.from_numpy(q)
+    tk = torch.from_numpy(np.repeat(k, Hq // Hkv, axis=1))
+    tv = torch.from_numpy(np.repeat(v, Hq // Hkv, axis=1))
+    ii = torch.arange(Sq).view(Sq, 1)
+    jj = torch.arange(Sk).view(1, Sk)
+    for causal in (True, False):
+        keep = (jj <= ii + (Sk - Sq)) if causal else torch.ones(Sq, Sk, dtype=torch.bool)
+        ref = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, attn_mask=keep)
+        logits = (tq @ tk.transpose(-1, -2) / math.sqrt(D)).masked_fill(~keep, float("-inf"))
+        ref_lse = torch.logsumexp(logits, dim=-1)
+        o, lse = orc.attention_qk(q, k, v, causal)
+        assert np.allclose(o, ref.numpy(), rtol=0, atol=1e-12)
+        assert np.allclose(lse, ref_lse.numpy(), rtol=0, atol=1e-12)
+
+
+def check_qk_edges(orc):
+    """One causal query sees every key; a causal query with no visible key is
+    rejected; the per-row entry agrees with the whole-tensor entry."""
+    r = _rng(13)
+    q = r.normal(size=(1, 2, 1, 8))
+    k = r.normal(size=(1, 1, 20, 8))
+    v = r.normal(size=(1, 1, 20, 8))
+    oc, lc = orc.attention_qk(q, k, v, True)
+    on, ln = orc.attention_qk(q, k, v, False)
+    assert np.array_equal(oc, on) and np.array_equal(lc, ln)
+    try:
+        orc.attention_qk(r.normal(size=(1, 2, 21, 8)), k, v, True)
+    except ValueError:
+        pass
+    else:
+        raise AssertionError("causal Sq > Sk accepted")
+    q2 = r.normal(size=(1, 2, 9, 8))
+    o, lse = orc.attention_qk(q2, k, v, True)
+    pos = np.array([0, 4, 8])
+    o2, l2 = orc.attention_rows_qk(q2[0, 1, pos], pos, k[0, 0], v[0, 0], 9, True)
+    assert np.array_equal(o2, o[0, 1, pos]) and np.array_equal(l2, lse[0, 1, pos])
+
+
 ALL_CHECKS = [check_golden, check_row_sums, check_constant_v, check_zero_query,
               check_first_causal_row, check_permutation, check_key_shift,
-              check_hard_attention, check_gqa, check_library, check_rows_api]
+              check_hard_attention, check_gqa, check_library, check_rows_api,
+              check_qk_suffix, check_qk_library, check_qk_edges]

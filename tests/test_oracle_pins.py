@@ -33,6 +33,16 @@ MUTATIONS = [
     ("value rows read in reverse", "v[j * D + d]", "v[(n_keys - 1 - j) * D + d]"),
     ("probabilities not normalised", "p_out[j] /= l;", "p_out[j] /= 1.0;"),
     ("query/key operand index swapped", "q[d] * k[j * D + d]", "q[d] * k[j * D + (D - 1 - d)]"),
+    # the different-length (Sq, Sk) entries
+    ("causal window aligned top-left", "const int64_t last = i + (Sk - Sq);",
+     "const int64_t last = i;"),
+    ("causal offset sign flipped", "const int64_t last = i + (Sk - Sq);",
+     "const int64_t last = i + (Sq - Sk);"),
+    ("Sq/Sk weights not normalised", "o[d] /= sum;", "o[d] /= 1.0;"),
+    ("Sq/Sk LSE drops the max term", "*lse = mx + log(sum);", "*lse = log(sum);"),
+    ("Sq/Sk value rows shifted", "o[d] += scratch[j] * v[D * j + d];",
+     "o[d] += scratch[j] * v[D * ((j + 1) % nk) + d];"),
+    ("Sq/Sk scale dropped", "pow((double)D, -0.5)", "1.0"),
 ]
 
 
