@@ -43,6 +43,8 @@ def load() -> ctypes.CDLL:
     vp, i, u64, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_uint64, ctypes.c_size_t
     lib.attn_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, vp]
     lib.attn_fwd.restype = i
+    lib.attn_fwd_qk.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, i, vp]
+    lib.attn_fwd_qk.restype = i
     lib.attn_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, vp]
     lib.attn_fwd_noalloc.restype = i
     lib.attn_fwd_host.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, vp, sz, vp]
@@ -88,18 +90,19 @@ def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = T
              o: torch.Tensor | None = None, lse: torch.Tensor | None = None, stream=None):
     """O, LSE = attention(Q, K, V) on the GPU through the C ABI.
 
-    q: [B,Hq,S,D] fp16; k, v: [B,Hkv,S,D] fp16 (contiguous, on the current
-    device).  Returns (o [B,Hq,S,D] fp16, lse [B,Hq,S] fp32); o / lse may be
-    passed in preallocated.  Asynchronous on ``stream`` (default: the current
-    torch stream).
+    q: [B,Hq,Sq,D] fp16; k, v: [B,Hkv,Sk,D] fp16 (contiguous, on the current
+    device).  Returns (o [B,Hq,Sq,D] fp16, lse [B,Hq,Sq] fp32); o / lse may be
+    passed in preallocated.  Sq == Sk calls attn_fwd, otherwise attn_fwd_qk
+    (causal window aligned at the bottom right, Sq <= Sk).  Asynchronous on
+    ``stream`` (default: the current torch stream).
     """
     lib = load()
     _check_dev(q, "q", torch.float16)
     _check_dev(k, "k", torch.float16)
     _check_dev(v, "v", torch.float16)
     B, Hq, S, D = q.shape
-    Hkv = k.shape[1]
-    if tuple(k.shape) != (B, Hkv, S, D) or tuple(v.shape) != tuple(k.shape):
+    Hkv, Sk = k.shape[1], k.shape[2]
+    if tuple(k.shape) != (B, Hkv, Sk, D) or tuple(v.shape) != tuple(k.shape):
         raise ValueError("shape mismatch: q %s k %s v %s" % (tuple(q.shape), tuple(k.shape),
                                                              tuple(v.shape)))
     if o is None:
@@ -108,10 +111,15 @@ def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = T
         lse = torch.empty((B, Hq, S), dtype=torch.float32, device=q.device)
     _check_dev(o, "o", torch.float16)
     _check_dev(lse, "lse", torch.float32)
-    st = lib.attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
-                      B, Hq, Hkv, S, D, int(bool(causal)), _stream_ptr(stream))
+    if Sk == S:
+        st = lib.attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                          B, Hq, Hkv, S, D, int(bool(causal)), _stream_ptr(stream))
+    else:
+        st = lib.attn_fwd_qk(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                             lse.data_ptr(), B, Hq, Hkv, S, Sk, D, int(bool(causal)),
+                             _stream_ptr(stream))
     if st != ATTN_OK:
-        raise AttnError(st, "attn_fwd")
+        raise AttnError(st, "attn_fwd" if Sk == S else "attn_fwd_qk")
     return o, lse
 
 

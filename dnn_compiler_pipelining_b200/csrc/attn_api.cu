@@ -152,9 +152,13 @@ bool encode_rows_map(CUtensorMap* map, const void* base, uint64_t rows, int D,
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-attn_status validate_sizes(int B, int Hq, int Hkv, int S, int D) {
-  if (B < 1 || Hq < 1 || Hkv < 1 || S < 1 || D < 1) return ATTN_ERR_SHAPE;
+attn_status validate_sizes(int B, int Hq, int Hkv, int S, int D, int Sk = -1, int causal = 0) {
+  if (Sk < 0) Sk = S;
+  if (B < 1 || Hq < 1 || Hkv < 1 || S < 1 || Sk < 1 || D < 1) return ATTN_ERR_SHAPE;
   if (Hq % Hkv != 0) return ATTN_ERR_SHAPE;
+  // a causal query with no visible key (Sq > Sk) has no softmax
+  if (causal && S > Sk) return ATTN_ERR_SHAPE;
+  if (static_cast<int64_t>(B) * Hkv * Sk >= (int64_t(1) << 31)) return ATTN_ERR_SHAPE;
   if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
   // row indices are 32-bit signed in the kernel and in TMA coordinates
   const int64_t q_rows = static_cast<int64_t>(B) * Hq * S;
@@ -165,6 +169,30 @@ attn_status validate_sizes(int B, int Hq, int Hkv, int S, int D) {
 
 size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
+// Kernel parameters of one call (Sq query rows over Sk keys).
+FwdParams make_params(void* o, float* lse, int B, int Hq, int Hkv, int Sq, int Sk, int D,
+                      int causal) {
+  FwdParams p;
+  p.o = static_cast<__half*>(o);
+  p.lse = lse;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.S = Sq;
+  p.Sk = Sk;
+  p.causal = causal ? 1 : 0;
+  p.off = causal ? Sk - Sq : 0;
+  p.n_qb = (Sq + kBlockM - 1) / kBlockM;
+  p.n_kb = (Sk + kBlockN - 1) / kBlockN;
+  p.s_tail = Sq - (p.n_qb - 1) * kBlockM;
+  p.n_qb2 = (p.n_qb + 1) / 2;
+  p.group = Hq / Hkv;
+  p.n_items = B * Hq * p.n_qb2;
+  p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
+  p.timeout_ns = g_timeout_ns.load();
+  return p;
+}
+
 // Tensor maps of one call: Q and V in 128-row boxes, K in 64-row boxes (the
 // pair pass loads half a key block per CTA) and 128-row boxes (redo pass).
 struct CallMaps {
@@ -172,9 +200,9 @@ struct CallMaps {
 };
 
 bool encode_call_maps(CallMaps* m, const void* q, const void* k, const void* v, int B, int Hq,
-                      int Hkv, int S, int D) {
-  const uint64_t q_rows = static_cast<uint64_t>(B) * Hq * S;
-  const uint64_t kv_rows = static_cast<uint64_t>(B) * Hkv * S;
+                      int Hkv, int Sq, int Sk, int D) {
+  const uint64_t q_rows = static_cast<uint64_t>(B) * Hq * Sq;
+  const uint64_t kv_rows = static_cast<uint64_t>(B) * Hkv * Sk;
   return encode_rows_map(&m->q, q, q_rows, D) && encode_rows_map(&m->k, k, kv_rows, D) &&
          encode_rows_map(&m->k_half, k, kv_rows, D, kBlockM / 2) &&
          encode_rows_map(&m->v, v, kv_rows, D);
@@ -185,8 +213,8 @@ bool encode_call_maps(CallMaps* m, const void* q, const void* k, const void* v, 
 template <int kD>
 attn_status launch_passes_d(const CallMaps& m, const FwdParams& p, int dev, cudaStream_t cs) {
   const int sms = g_dev_sms[dev];
-  // the pair kernel takes D = 128 and whole 128-row blocks only
-  if (kPairFusedPass && kD == 128 && p.s_tail == kBlockM) {
+  // the pair kernel takes D = 128, Sq == Sk and whole 128-row blocks only
+  if (kPairFusedPass && kD == 128 && p.S == p.Sk && p.s_tail == kBlockM) {
     const int pairs = p.n_items < g_dev_pairs[dev] ? p.n_items : g_dev_pairs[dev];
     pair::attn_fwd_pair_kernel<<<2 * pairs, pair::kThreads, pair_smem_bytes(), cs>>>(
         m.q, m.k_half, m.v, p);
@@ -237,10 +265,10 @@ uint64_t attn_set_wait_timeout_ns(uint64_t ns) {
   return g_timeout_ns.exchange(ns);
 }
 
-attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
-                     int Hq, int Hkv, int S, int D, int causal, void* stream) {
+attn_status attn_fwd_qk(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                        int Hq, int Hkv, int Sq, int Sk, int D, int causal, void* stream) {
   if (!q || !k || !v || !o || !lse) return ATTN_ERR_NULL;
-  attn_status st = validate_sizes(B, Hq, Hkv, S, D);
+  attn_status st = validate_sizes(B, Hq, Hkv, Sq, D, Sk, causal);
   if (st != ATTN_OK) return st;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
     return ATTN_ERR_ALIGN;
@@ -249,29 +277,19 @@ attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float
   if (st != ATTN_OK) return st;
 
   CallMaps maps;
-  if (!encode_call_maps(&maps, q, k, v, B, Hq, Hkv, S, D)) return ATTN_ERR_CUDA;
-
-  FwdParams p;
-  p.o = static_cast<__half*>(o);
-  p.lse = lse;
-  p.B = B;
-  p.Hq = Hq;
-  p.Hkv = Hkv;
-  p.S = S;
-  p.causal = causal ? 1 : 0;
-  p.n_qb = (S + kBlockM - 1) / kBlockM;
-  p.s_tail = S - (p.n_qb - 1) * kBlockM;
-  p.n_qb2 = (p.n_qb + 1) / 2;
-  p.group = Hq / Hkv;
-  p.n_items = B * Hq * p.n_qb2;
-  p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
-  p.timeout_ns = g_timeout_ns.load();
+  if (!encode_call_maps(&maps, q, k, v, B, Hq, Hkv, Sq, Sk, D)) return ATTN_ERR_CUDA;
+  FwdParams p = make_params(o, lse, B, Hq, Hkv, Sq, Sk, D, causal);
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   p.redo = redo_list(dev, cs);
   if (!p.redo) return ATTN_ERR_CUDA;
   p.redo_capacity = kRedoCapacity;
 
   return launch_passes(maps, p, D, dev, cs);
+}
+
+attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                     int Hq, int Hkv, int S, int D, int causal, void* stream) {
+  return attn_fwd_qk(q, k, v, o, lse, B, Hq, Hkv, S, S, D, causal, stream);
 }
 
 size_t attn_fwd_host_workspace_bytes(int B, int Hq, int Hkv, int S, int D) {
@@ -430,23 +448,9 @@ extern "C" attn_status attn_fwd_noalloc(const void* q, const void* k, const void
   if (!scratch) return ATTN_ERR_CUDA;
 
   CallMaps maps;
-  if (!encode_call_maps(&maps, q, k, v, B, Hq, Hkv, S, D)) return ATTN_ERR_CUDA;
+  if (!encode_call_maps(&maps, q, k, v, B, Hq, Hkv, S, S, D)) return ATTN_ERR_CUDA;
 
-  FwdParams p;
-  p.o = static_cast<__half*>(o);
-  p.lse = lse;
-  p.B = B;
-  p.Hq = Hq;
-  p.Hkv = Hkv;
-  p.S = S;
-  p.causal = causal ? 1 : 0;
-  p.n_qb = n_qb;
-  p.s_tail = S - (n_qb - 1) * kBlockM;
-  p.n_qb2 = n_qb2;
-  p.group = Hq / Hkv;
-  p.n_items = static_cast<int>(n_items);
-  p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
-  p.timeout_ns = g_timeout_ns.load();
+  FwdParams p = make_params(o, lse, B, Hq, Hkv, S, S, D, causal);
   p.redo = scratch;
   p.redo_capacity = kNoAllocMaxItems;  // >= n_items: the list cannot overflow
   cudaStream_t cs = static_cast<cudaStream_t>(stream);

@@ -92,11 +92,14 @@ constexpr int kRedoHeaderWords = 4;
 struct FwdParams {
   __half* o;
   float* lse;
-  int B, Hq, Hkv, S;
+  int B, Hq, Hkv, S;  // S: query rows per head (Sq)
+  int Sk;             // keys per kv head
   int causal;
-  int n_items;       // B * Hq * n_qb2
-  int n_qb;          // ceil(S / 128) row (and key) blocks
-  int s_tail;        // rows (keys) in the last block, 1..128
+  int off;            // causal window offset Sk - Sq: query i sees keys j <= i + off
+  int n_items;        // B * Hq * n_qb2
+  int n_qb;           // ceil(S / 128) row blocks
+  int n_kb;           // ceil(Sk / 128) key blocks
+  int s_tail;         // rows in the last row block, 1..128
   int n_qb2;         // ceil(n_qb / 2) items per (batch, head)
   int group;         // Hq / Hkv
   float scale_log2;  // log2(e) / sqrt(D)
@@ -171,11 +174,16 @@ __device__ __forceinline__ Item decode_item(const FwdParams& p, int id) {
   it.hq = it.g * p.group + rem % p.group;
   const bool b_active = 2 * it.qb2 + 1 < p.n_qb;
   if (p.causal) {
-    it.n_kv[0] = 2 * it.qb2 + 1;
-    it.n_kv[1] = b_active ? 2 * it.qb2 + 2 : 0;
+    // the tile's last row sees keys up to row + off; no further key block
+#pragma unroll
+    for (int x = 0; x < 2; ++x) {
+      const int last_row = min((2 * it.qb2 + x) * kBlockM + kBlockM - 1, p.S - 1);
+      it.n_kv[x] = min(p.n_kb, (last_row + p.off) / kBlockN + 1);
+    }
+    if (!b_active) it.n_kv[1] = 0;
   } else {
-    it.n_kv[0] = p.n_qb;
-    it.n_kv[1] = b_active ? p.n_qb : 0;
+    it.n_kv[0] = p.n_kb;
+    it.n_kv[1] = b_active ? p.n_kb : 0;
   }
   it.n_blocks = it.n_kv[1] > it.n_kv[0] ? it.n_kv[1] : it.n_kv[0];
   return it;
@@ -359,7 +367,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                  once);
             }
           }
-          const int kv_row = (it.b * p.Hkv + it.g) * p.S;
+          const int kv_row = (it.b * p.Hkv + it.g) * p.Sk;
           for (int j = 0; j < it.n_blocks; ++j, ++rc) {
             const int depth = is_v ? kStagesV : kStagesK;
             const int st = rc % depth;
@@ -553,8 +561,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         const Item it = decode_item(p, item);
         const int n_x = it.n_kv[x];
         if (n_x == 0) continue;
-        const int diag = p.causal ? n_x - 1 : -1;
-        const int tail_blk = p.causal ? -1 : n_x - 1;
+        // the last key this row sees: row + off (causal), and never past Sk
+        // (a ragged last key block reads the next head's rows, or zero fill
+        // past the tensor); rows past S are computed but not stored
+        const int i_row = (2 * it.qb2 + x) * kBlockM + r;
+        const int key_lim = p.causal ? min(i_row + p.off, p.Sk - 1) : p.Sk - 1;
+        // key_lim grows with the lane, so from this block on (warp-uniform)
+        // some lane of the warp has keys to mask
+        const int j_mask = (__shfl_sync(0xffffffffu, key_lim, 0) + 1) / kBlockN;
         float m_use = -INFINITY;
         float l = 0.f;
         bool ok = true;
@@ -573,12 +587,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_wait_ld();
 #pragma unroll
           for (int c = 0; c < 4; ++c) reg_dep32(&u[c * 32]);
-          // causal: the diagonal block keeps keys <= row.  Non-causal: a
-          // ragged last block keeps its first s_tail keys (the rows past S
-          // belong to the next head or lie past the tensor, zero-filled);
-          // with the causal mask the diagonal block already hides them.
-          if (j == diag || (j == tail_blk && p.s_tail < kBlockN)) {
-            const int lim = j == diag ? r : p.s_tail - 1;
+          // keys past the row's limit -> -inf (the causal diagonal, a
+          // ragged last key block)
+          if (j >= j_mask) {
+            const int lim = key_lim - j * kBlockN;
 #pragma unroll
             for (int c = 0; c < 128; ++c)
               if (c > lim) u[c] = 0xff800000u;  // -inf

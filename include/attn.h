@@ -83,6 +83,21 @@ attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float
                      int B, int Hq, int Hkv, int S, int D, int causal, void* stream);
 
 /*
+ * attn_fwd_qk -- attn_fwd with Sq query rows over Sk keys (Sq != Sk allowed).
+ * Not in the pages, which evaluate Sq == Sk only: needed for a prefill over a
+ * cached key prefix (Sq < Sk) and for non-causal cross attention.
+ *   q, o: [B, Hq, Sq, D]; k, v: [B, Hkv, Sk, D]; lse: [B, Hq, Sq].
+ *   causal: query i sees keys j <= i + (Sk - Sq) (aligned at the bottom right:
+ *   the last query sees every key); requires Sq <= Sk (ATTN_ERR_SHAPE
+ *   otherwise, as a query would see no key).  Non-causal: any Sq, Sk >= 1.
+ * Everything else (pointers, alignment, D, streams, the two launches, errors)
+ * is as for attn_fwd, which is attn_fwd_qk with Sq == Sk == S.
+ */
+attn_status attn_fwd_qk(const void* q, const void* k, const void* v, void* o, float* lse,
+                        int B, int Hq, int Hkv, int Sq, int Sk, int D, int causal,
+                        void* stream);
+
+/*
  * attn_fwd_host_workspace_bytes -- size in bytes of the device workspace that
  * attn_fwd_host needs for these sizes (Q, K, V, O and LSE, each rounded up to
  * 256 bytes).  Returns 0 for invalid sizes.

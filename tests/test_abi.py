@@ -65,6 +65,20 @@ def test_validation_before_launch(lib):
     assert call(lib, lse=FAKE + 4) == ALIGN
 
 
+def test_qk_validation_before_launch(lib):
+    lib.attn_fwd_qk.argtypes = [ctypes.c_void_p] * 5 + [ctypes.c_int] * 7 + [ctypes.c_void_p]
+
+    def qk(Sq, Sk, causal, D=128):
+        return lib.attn_fwd_qk(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 4, 2, Sq, Sk, D, causal, None)
+
+    assert qk(300, 200, 1) == SHAPE         # a causal query would see no key
+    assert qk(0, 200, 0) == SHAPE
+    assert qk(200, 0, 0) == SHAPE
+    assert qk(100, 200, 1, D=96) == UNSUP
+    assert qk(100, 200, 1) in (CUDA, UNSUP)   # well-formed: reaches the runtime
+    assert qk(300, 200, 0) in (CUDA, UNSUP)   # non-causal Sq > Sk is allowed
+
+
 def test_valid_call_without_gpu_fails_loudly(lib):
     # well-formed arguments reach the CUDA runtime, which has no device here
     assert call(lib) in (CUDA, UNSUP)

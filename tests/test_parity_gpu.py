@@ -102,6 +102,56 @@ def test_d64_sampled(causal):
     parity.sampled_check(q, k, v, o, lse, causal, n_random=512, seed=31)
 
 
+# Sq query rows over Sk keys (attn_fwd_qk); causal windows aligned bottom-right
+QK = [(1, 4, 2, 1, 513), (2, 4, 2, 77, 300), (1, 8, 2, 128, 1000), (1, 6, 3, 257, 1024),
+      (2, 4, 1, 300, 300)]
+
+
+def _qk_inputs(B, Hq, Hkv, Sq, Sk, D, seed, qk_std=1.0):
+    q, _, _ = make_qkv(B, Hq, Hkv, Sq, D, seed=seed, qk_std=qk_std, device="cuda")
+    _, k, v = make_qkv(B, Hq, Hkv, Sk, D, seed=seed + 100, qk_std=qk_std, device="cuda")
+    return q, k, v
+
+
+def _qk_check(q, k, v, causal, what):
+    o, lse = parity.run_gpu(q, k, v, causal)
+    o_ref, lse_ref = parity.oracle.attention_qk(q.cpu().double().numpy(), k.cpu().double().numpy(),
+                                                v.cpu().double().numpy(), causal)
+    parity.assert_close(o.cpu().double().numpy(), o_ref, lse.cpu().double().numpy(), lse_ref, what)
+
+
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("B,Hq,Hkv,Sq,Sk", QK)
+def test_qk_full(B, Hq, Hkv, Sq, Sk, causal):
+    q, k, v = _qk_inputs(B, Hq, Hkv, Sq, Sk, 128, seed=37)
+    _qk_check(q, k, v, causal, "Sq%d Sk%d causal=%d" % (Sq, Sk, causal))
+
+
+def test_qk_noncausal_more_queries_than_keys():
+    q, k, v = _qk_inputs(1, 4, 2, 500, 130, 128, seed=43)
+    _qk_check(q, k, v, False, "Sq500 Sk130")
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_qk_stress_and_d64(causal):
+    q, k, v = _qk_inputs(1, 8, 2, 100, 700, 128, seed=47, qk_std=4.0)
+    _qk_check(q, k, v, causal, "stress Sq100 Sk700")
+    q, k, v = _qk_inputs(1, 4, 2, 200, 450, 64, seed=53)
+    _qk_check(q, k, v, causal, "D64 Sq200 Sk450")
+
+
+def test_qk_prefill_over_long_prefix():
+    """64 new queries over 8192 cached keys (causal, bottom-right)."""
+    q, k, v = _qk_inputs(2, 32, 8, 64, 8192, 128, seed=59)
+    _qk_check(q, k, v, True, "Sq64 Sk8192")
+
+
+def test_qk_causal_more_queries_than_keys_rejected():
+    q, k, v = _qk_inputs(1, 4, 2, 300, 200, 128, seed=61)
+    with pytest.raises(attn.AttnError):
+        attn.attn_fwd(q, k, v, True)
+
+
 def test_llama3_8b_s512_b1_full():
     w = WORKLOADS["llama3-8b-s512-b1"]
     parity.full_check(w["B"], w["Hq"], w["Hkv"], w["S"], w["D"], w["causal"], seed=0)
