@@ -152,6 +152,30 @@ bool encode_rows_map(CUtensorMap* map, const void* base, uint64_t rows, int D,
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Streams of attn_fwd_host's copy / compute pipeline, created once per device
+// (non-blocking, so they do not serialize with the legacy default stream).
+constexpr int kHostChunks = 8;
+struct HostPipe {
+  cudaStream_t up, comp, down;
+};
+HostPipe* g_host_pipe[kMaxDevices];
+std::mutex g_host_pipe_mutex;
+
+HostPipe* host_pipe(int dev) {
+  std::lock_guard<std::mutex> lock(g_host_pipe_mutex);
+  if (!g_host_pipe[dev]) {
+    HostPipe* hp = new HostPipe;
+    if (cudaStreamCreateWithFlags(&hp->up, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaStreamCreateWithFlags(&hp->comp, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaStreamCreateWithFlags(&hp->down, cudaStreamNonBlocking) != cudaSuccess) {
+      delete hp;
+      return nullptr;
+    }
+    g_host_pipe[dev] = hp;
+  }
+  return g_host_pipe[dev];
+}
+
 attn_status validate_sizes(int B, int Hq, int Hkv, int S, int D, int Sk = -1, int causal = 0) {
   if (Sk < 0) Sk = S;
   if (B < 1 || Hq < 1 || Hkv < 1 || S < 1 || Sk < 1 || D < 1) return ATTN_ERR_SHAPE;
@@ -270,7 +294,8 @@ attn_status attn_fwd_qk(const void* q, const void* k, const void* v, void* o, fl
   if (!q || !k || !v || !o || !lse) return ATTN_ERR_NULL;
   attn_status st = validate_sizes(B, Hq, Hkv, Sq, D, Sk, causal);
   if (st != ATTN_OK) return st;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u) != 0)
     return ATTN_ERR_ALIGN;
   int dev = 0;
   st = device_setup(&dev);
@@ -323,26 +348,83 @@ attn_status attn_fwd_host(const void* q_h, const void* k_h, const void* v_h, voi
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return ATTN_ERR_ALIGN;
   const size_t need = attn_fwd_host_workspace_bytes(B, Hq, Hkv, S, D);
   if (workspace_bytes < need) return ATTN_ERR_WORKSPACE;
-  const size_t qb = static_cast<size_t>(B) * Hq * S * D * 2;
-  const size_t kvb = static_cast<size_t>(B) * Hkv * S * D * 2;
-  const size_t lb = static_cast<size_t>(B) * Hq * S * 4;
+  int dev = 0;
+  st = device_setup(&dev);
+  if (st != ATTN_OK) return st;
+  // per batch element (BHSD: each b is one contiguous slice of every tensor)
+  const size_t qb1 = static_cast<size_t>(Hq) * S * D * 2;
+  const size_t kvb1 = static_cast<size_t>(Hkv) * S * D * 2;
+  const size_t lb1 = static_cast<size_t>(Hq) * S * 4;
   char* w = static_cast<char*>(workspace);
   char* dq = w;
-  char* dk = dq + round256(qb);
-  char* dv = dk + round256(kvb);
-  char* dout = dv + round256(kvb);
-  float* dl = reinterpret_cast<float*>(dout + round256(qb));
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (cudaMemcpyAsync(dq, q_h, qb, cudaMemcpyHostToDevice, s) != cudaSuccess ||
-      cudaMemcpyAsync(dk, k_h, kvb, cudaMemcpyHostToDevice, s) != cudaSuccess ||
-      cudaMemcpyAsync(dv, v_h, kvb, cudaMemcpyHostToDevice, s) != cudaSuccess)
-    return ATTN_ERR_CUDA;
-  st = attn_fwd(dq, dk, dv, dout, dl, B, Hq, Hkv, S, D, causal, stream);
-  if (st != ATTN_OK) return st;
-  if (cudaMemcpyAsync(o_h, dout, qb, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
-      cudaMemcpyAsync(lse_h, dl, lb, cudaMemcpyDeviceToHost, s) != cudaSuccess)
-    return ATTN_ERR_CUDA;
-  return attn_device_status(stream, nullptr);
+  char* dk = dq + round256(qb1 * B);
+  char* dv = dk + round256(kvb1 * B);
+  char* dout = dv + round256(kvb1 * B);
+  char* dl = dout + round256(qb1 * B);
+  const char* hq = static_cast<const char*>(q_h);
+  const char* hk = static_cast<const char*>(k_h);
+  const char* hv = static_cast<const char*>(v_h);
+  char* ho = static_cast<char*>(o_h);
+  char* hl = reinterpret_cast<char*>(lse_h);
+
+  // Three-stage pipeline over chunks of the batch on this device's copy /
+  // compute streams: uploads of chunk c+1 and downloads of chunk c-1 overlap
+  // the kernels of chunk c (and each other: host links are full duplex).
+  // Events order the stages per chunk and the whole call after the work
+  // already on `stream`; `stream` waits for the last download.
+  HostPipe* hp = host_pipe(dev);
+  if (!hp) return ATTN_ERR_CUDA;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  const int n_chunks = B < kHostChunks ? B : kHostChunks;
+  cudaEvent_t ev[1 + 2 * kHostChunks + 1];
+  int n_ev = 0;
+  auto fail = [&](attn_status e) {
+    cudaStreamSynchronize(hp->up);
+    cudaStreamSynchronize(hp->comp);
+    cudaStreamSynchronize(hp->down);
+    for (int i = 0; i < n_ev; ++i) cudaEventDestroy(ev[i]);
+    return e;
+  };
+  for (int i = 0; i < 2 + 2 * n_chunks; ++i) {
+    if (cudaEventCreateWithFlags(&ev[i], cudaEventDisableTiming) != cudaSuccess)
+      return fail(ATTN_ERR_CUDA);
+    ++n_ev;
+  }
+  cudaEvent_t ev_start = ev[0], ev_end = ev[1 + 2 * n_chunks];
+  if (cudaEventRecord(ev_start, cs) != cudaSuccess ||
+      cudaStreamWaitEvent(hp->up, ev_start, 0) != cudaSuccess)
+    return fail(ATTN_ERR_CUDA);
+  for (int c = 0; c < n_chunks; ++c) {
+    const int b0 = static_cast<int>(static_cast<int64_t>(B) * c / n_chunks);
+    const int b1 = static_cast<int>(static_cast<int64_t>(B) * (c + 1) / n_chunks);
+    const int nb = b1 - b0;
+    cudaEvent_t up_done = ev[1 + 2 * c], comp_done = ev[2 + 2 * c];
+    if (cudaMemcpyAsync(dq + qb1 * b0, hq + qb1 * b0, qb1 * nb, cudaMemcpyHostToDevice,
+                        hp->up) != cudaSuccess ||
+        cudaMemcpyAsync(dk + kvb1 * b0, hk + kvb1 * b0, kvb1 * nb, cudaMemcpyHostToDevice,
+                        hp->up) != cudaSuccess ||
+        cudaMemcpyAsync(dv + kvb1 * b0, hv + kvb1 * b0, kvb1 * nb, cudaMemcpyHostToDevice,
+                        hp->up) != cudaSuccess ||
+        cudaEventRecord(up_done, hp->up) != cudaSuccess ||
+        cudaStreamWaitEvent(hp->comp, up_done, 0) != cudaSuccess)
+      return fail(ATTN_ERR_CUDA);
+    st = attn_fwd(dq + qb1 * b0, dk + kvb1 * b0, dv + kvb1 * b0, dout + qb1 * b0,
+                  reinterpret_cast<float*>(dl + lb1 * b0), nb, Hq, Hkv, S, D, causal, hp->comp);
+    if (st != ATTN_OK) return fail(st);
+    if (cudaEventRecord(comp_done, hp->comp) != cudaSuccess ||
+        cudaStreamWaitEvent(hp->down, comp_done, 0) != cudaSuccess ||
+        cudaMemcpyAsync(ho + qb1 * b0, dout + qb1 * b0, qb1 * nb, cudaMemcpyDeviceToHost,
+                        hp->down) != cudaSuccess ||
+        cudaMemcpyAsync(hl + lb1 * b0, dl + lb1 * b0, lb1 * nb, cudaMemcpyDeviceToHost,
+                        hp->down) != cudaSuccess)
+      return fail(ATTN_ERR_CUDA);
+  }
+  if (cudaEventRecord(ev_end, hp->down) != cudaSuccess ||
+      cudaStreamWaitEvent(cs, ev_end, 0) != cudaSuccess)
+    return fail(ATTN_ERR_CUDA);
+  st = attn_device_status(stream, nullptr);
+  for (int i = 0; i < n_ev; ++i) cudaEventDestroy(ev[i]);
+  return st;
 }
 
 }  // extern "C"
@@ -435,7 +517,8 @@ extern "C" attn_status attn_fwd_noalloc(const void* q, const void* k, const void
   if (!q || !k || !v || !o || !lse) return ATTN_ERR_NULL;
   attn_status st = validate_sizes(B, Hq, Hkv, S, D);
   if (st != ATTN_OK) return st;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u) != 0)
     return ATTN_ERR_ALIGN;
   const int n_qb = (S + kBlockM - 1) / kBlockM;
   const int n_qb2 = (n_qb + 1) / 2;

@@ -53,7 +53,7 @@ typedef enum attn_status {
   ATTN_OK = 0,
   ATTN_ERR_NULL = 1,           /* a required pointer is NULL */
   ATTN_ERR_SHAPE = 2,          /* B,Hq,Hkv,S < 1, Hq % Hkv != 0, or a size overflows */
-  ATTN_ERR_ALIGN = 3,          /* a device pointer is not 16-byte aligned */
+  ATTN_ERR_ALIGN = 3,          /* q, k, v, o not 16-byte aligned, or lse not 4-byte aligned */
   ATTN_ERR_UNSUPPORTED = 4,    /* D not 64 or 128, or not an sm_100 device */
   ATTN_ERR_CUDA = 5,           /* a CUDA runtime / driver call failed */
   ATTN_ERR_DEVICE_TIMEOUT = 6, /* a kernel wait ran out; results are invalid */
@@ -66,7 +66,7 @@ typedef enum attn_status {
  *   q   : device, fp16 [B, Hq, S, D], 16-byte aligned, read only.
  *   k, v: device, fp16 [B, Hkv, S, D], 16-byte aligned, read only.
  *   o   : device, fp16 [B, Hq, S, D], 16-byte aligned, written.
- *   lse : device, fp32 [B, Hq, S], 16-byte aligned, written (must not be NULL).
+ *   lse : device, fp32 [B, Hq, S], 4-byte aligned, written (must not be NULL).
  *   B, Hq, Hkv, S, D: sizes; Hq % Hkv == 0; D == 64 or 128; any S >= 1 (a
  *   last block of fewer than 128 rows is computed with the keys past S
  *   masked).
@@ -108,10 +108,14 @@ size_t attn_fwd_host_workspace_bytes(int B, int Hq, int Hkv, int S, int D);
  * attn_fwd_host -- the same operation on HOST buffers, for callers whose data
  * live in CPU memory.  q_h, k_h, v_h (fp16, layouts as above) are copied into
  * the caller's device workspace, attn_fwd runs there, and O and LSE are
- * copied back into o_h (fp16) and lse_h (fp32).  All copies and the kernel
- * are enqueued on `stream`, and the call synchronizes the stream before it
- * returns, so the host buffers hold the results on ATTN_OK.  Host buffers may
- * be pageable or pinned (pinned copies run asynchronously and faster).
+ * copied back into o_h (fp16) and lse_h (fp32).  The work runs as a pipeline
+ * over up to 8 chunks of the batch on the library's own per-device streams
+ * (uploads, kernels, downloads), so copies of one chunk overlap the kernels
+ * of another; it starts after the work already enqueued on `stream`, `stream`
+ * waits for it, and the call synchronizes `stream` before it returns, so the
+ * host buffers hold the results on ATTN_OK.  Host buffers may be pageable or
+ * pinned (pinned copies run asynchronously and faster).  The library creates
+ * those three streams on its first call for each device and keeps them.
  *   workspace: device, >= attn_fwd_host_workspace_bytes(...) bytes, 256-byte
  *              aligned; its contents are overwritten.
  * Also returns ATTN_ERR_DEVICE_TIMEOUT if the kernel reported one.

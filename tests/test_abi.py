@@ -62,7 +62,7 @@ def test_validation_before_launch(lib):
     assert call(lib, B=65536, Hq=1, Hkv=1, S=128) == SHAPE
     assert call(lib, B=64, Hq=64, Hkv=8, S=1 << 20) == SHAPE  # row index overflow
     assert call(lib, q=FAKE + 8) == ALIGN
-    assert call(lib, lse=FAKE + 4) == ALIGN
+    assert call(lib, lse=FAKE + 2) == ALIGN
 
 
 def test_qk_validation_before_launch(lib):

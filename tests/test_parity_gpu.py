@@ -222,13 +222,21 @@ def test_constant_v():
         assert (o.double() - c.double()).abs().max().item() <= parity.O_TOL
 
 
-def test_host_entry_matches_device_entry():
-    B, Hq, Hkv, S, D = 1, 8, 2, 512, 128
+@pytest.mark.parametrize("B,Hq,Hkv,S,D,pinned", [(1, 8, 2, 512, 128, True),
+                                                 (11, 4, 2, 384, 128, True),
+                                                 (3, 1, 1, 77, 64, True),
+                                                 (5, 2, 1, 200, 128, False)])
+def test_host_entry_matches_device_entry(B, Hq, Hkv, S, D, pinned):
+    """The host-buffer entry (a pipeline over up to 8 batch chunks on the
+    library's own streams) gives the device entry's bytes, including chunks
+    whose LSE slices start off a 16-byte boundary, and from pageable memory."""
     q, k, v = make_qkv(B, Hq, Hkv, S, D, seed=9, device="cuda")
     o, lse = parity.run_gpu(q, k, v, True)
-    qh, kh, vh = q.cpu().pin_memory(), k.cpu().pin_memory(), v.cpu().pin_memory()
-    oh = torch.empty_like(qh).pin_memory()
-    lh = torch.empty(B, Hq, S, dtype=torch.float32).pin_memory()
+    qh, kh, vh = q.cpu(), k.cpu(), v.cpu()
+    oh = torch.full_like(qh, float("nan"))
+    lh = torch.full((B, Hq, S), float("nan"), dtype=torch.float32)
+    if pinned:
+        qh, kh, vh, oh, lh = (t.pin_memory() for t in (qh, kh, vh, oh, lh))
     ws = torch.empty(attn.host_workspace_bytes(B, Hq, Hkv, S, D), dtype=torch.uint8, device="cuda")
     attn.attn_fwd_host(qh, kh, vh, oh, lh, True, ws)
     assert torch.equal(oh, o.cpu()) and torch.equal(lh, lse.cpu())
