@@ -154,7 +154,7 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 // Streams of attn_fwd_host's copy / compute pipeline, created once per device
 // (non-blocking, so they do not serialize with the legacy default stream).
-constexpr int kHostChunks = 8;
+constexpr int kHostChunks = 16;
 struct HostPipe {
   cudaStream_t up, comp, down;
 };

@@ -57,8 +57,10 @@ WORKLOADS = {
     "llama3-8b-s2048-b64": dict(B=64, Hq=32, Hkv=8, S=2048, D=128, causal=True),
     "llama3-70b-s8192-b64": dict(B=64, Hq=64, Hkv=8, S=8192, D=128, causal=True),
     "llama3-8b-s8192-b64": dict(B=64, Hq=32, Hkv=8, S=8192, D=128, causal=True),
-    # small case of the same kernel for profiler captures (Q alone exceeds L2)
+    # small cases of the same kernel for profiler captures (Q alone exceeds L2)
     "llama3-8b-s8192-b4": dict(B=4, Hq=32, Hkv=8, S=8192, D=128, causal=True),
+    "llama3-8b-s2048-b8": dict(B=8, Hq=32, Hkv=8, S=2048, D=128, causal=True),
+    "llama3-70b-s8192-b4": dict(B=4, Hq=64, Hkv=8, S=8192, D=128, causal=True),
 }
 
 

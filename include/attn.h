@@ -109,7 +109,7 @@ size_t attn_fwd_host_workspace_bytes(int B, int Hq, int Hkv, int S, int D);
  * live in CPU memory.  q_h, k_h, v_h (fp16, layouts as above) are copied into
  * the caller's device workspace, attn_fwd runs there, and O and LSE are
  * copied back into o_h (fp16) and lse_h (fp32).  The work runs as a pipeline
- * over up to 8 chunks of the batch on the library's own per-device streams
+ * over up to 16 chunks of the batch on the library's own per-device streams
  * (uploads, kernels, downloads), so copies of one chunk overlap the kernels
  * of another; it starts after the work already enqueued on `stream`, `stream`
  * waits for it, and the call synchronizes `stream` before it returns, so the

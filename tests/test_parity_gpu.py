@@ -227,7 +227,7 @@ def test_constant_v():
                                                  (3, 1, 1, 77, 64, True),
                                                  (5, 2, 1, 200, 128, False)])
 def test_host_entry_matches_device_entry(B, Hq, Hkv, S, D, pinned):
-    """The host-buffer entry (a pipeline over up to 8 batch chunks on the
+    """The host-buffer entry (a pipeline over up to 16 batch chunks on the
     library's own streams) gives the device entry's bytes, including chunks
     whose LSE slices start off a 16-byte boundary, and from pageable memory."""
     q, k, v = make_qkv(B, Hq, Hkv, S, D, seed=9, device="cuda")
