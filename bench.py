@@ -40,7 +40,8 @@ NOMINAL_DENSE_FP16_TFLOPS = 2250.0
 FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
 PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "attn_fwd_llama3-8b-s8192-b64.md")
 KERNEL_SOURCES = [os.path.join(ROOT, "dnn_compiler_pipelining_b200", "csrc", f)
-                  for f in ("attn_fwd_sm100.cuh", "ptx_sm100.cuh", "attn_api.cu")]
+                  for f in ("attn_fwd_sm100.cuh", "ptx_sm100.cuh", "attn_api.cu",
+                            "variant_table.inc")]
 
 
 def attn_flops(B, Hq, S, D, causal):

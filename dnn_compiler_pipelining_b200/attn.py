@@ -45,6 +45,14 @@ def load() -> ctypes.CDLL:
     lib.attn_fwd.restype = i
     lib.attn_fwd_qk.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, i, vp]
     lib.attn_fwd_qk.restype = i
+    lib.attn_fwd_variant.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, vp]
+    lib.attn_fwd_variant.restype = i
+    lib.attn_variant_count.argtypes = []
+    lib.attn_variant_count.restype = i
+    lib.attn_variant_name.argtypes = [i]
+    lib.attn_variant_name.restype = ctypes.c_char_p
+    lib.attn_variant_select.argtypes = [i, i, i, i, i, i, i]
+    lib.attn_variant_select.restype = i
     lib.attn_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, vp]
     lib.attn_fwd_noalloc.restype = i
     lib.attn_fwd_host.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, vp, sz, vp]
@@ -120,6 +128,49 @@ def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = T
                              _stream_ptr(stream))
     if st != ATTN_OK:
         raise AttnError(st, "attn_fwd" if Sk == S else "attn_fwd_qk")
+    return o, lse
+
+
+def variant_count() -> int:
+    """Number of compiled fused-pass variants."""
+    return int(load().attn_variant_count())
+
+
+def variant_name(variant: int) -> str | None:
+    name = load().attn_variant_name(int(variant))
+    return name.decode() if name is not None else None
+
+
+def variant_select(B: int, Hq: int, Hkv: int, Sq: int, Sk: int, D: int, causal: bool) -> int:
+    """The variant the library's measured table picks for these sizes (-1: invalid sizes).
+    Host-only: touches no device."""
+    return int(load().attn_variant_select(B, Hq, Hkv, Sq, Sk, D, int(bool(causal))))
+
+
+def attn_fwd_variant(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool,
+                     variant: int, o: torch.Tensor | None = None,
+                     lse: torch.Tensor | None = None, stream=None):
+    """attn_fwd with an explicit fused-pass variant (for the tuner and tests)."""
+    lib = load()
+    _check_dev(q, "q", torch.float16)
+    _check_dev(k, "k", torch.float16)
+    _check_dev(v, "v", torch.float16)
+    B, Hq, S, D = q.shape
+    Hkv, Sk = k.shape[1], k.shape[2]
+    if tuple(k.shape) != (B, Hkv, Sk, D) or tuple(v.shape) != tuple(k.shape):
+        raise ValueError("shape mismatch: q %s k %s v %s" % (tuple(q.shape), tuple(k.shape),
+                                                             tuple(v.shape)))
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, S), dtype=torch.float32, device=q.device)
+    _check_dev(o, "o", torch.float16)
+    _check_dev(lse, "lse", torch.float32)
+    st = lib.attn_fwd_variant(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                              lse.data_ptr(), B, Hq, Hkv, S, Sk, D, int(bool(causal)),
+                              int(variant), _stream_ptr(stream))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_fwd_variant")
     return o, lse
 
 

@@ -14,7 +14,8 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libattn_b200.so")
 SOURCES = [os.path.join(CSRC, "attn_api.cu")]
-DEPS = SOURCES + [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith(".cuh")] + \
+DEPS = SOURCES + [os.path.join(CSRC, f) for f in os.listdir(CSRC)
+                  if f.endswith(".cuh") or f.endswith(".inc")] + \
     [os.path.join(INCLUDE, "attn.h")]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")

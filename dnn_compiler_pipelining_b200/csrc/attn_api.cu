@@ -6,9 +6,11 @@
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
+#include <array>
 #include <atomic>
 #include <cmath>
 #include <cstdint>
+#include <cstdio>
 #include <map>
 #include <mutex>
 #include <utility>
@@ -83,6 +85,54 @@ size_t fwd_smem_bytes(int D = kHeadDim) {
 }
 size_t pair_smem_bytes() { return sizeof(pair::SharedPair); }
 
+// The fused-pass kernels of one head dimension, indexed by variant
+// (kEmuChoices[variant] FMA-pipe exponentials per 8 column pairs).
+using FwdKernel = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap,
+                           const FwdParams);
+template <int kD, int... kV>
+std::array<FwdKernel, sizeof...(kV)> fused_kernels(std::integer_sequence<int, kV...>) {
+  return {{&attn_fwd_kernel<0, kD, kEmuChoices[kV]>...}};
+}
+template <int kD>
+FwdKernel fused_kernel(int variant) {
+  static const std::array<FwdKernel, kNumVariants> table =
+      fused_kernels<kD>(std::make_integer_sequence<int, kNumVariants>{});
+  return table[variant];
+}
+
+// Measured choice of fused-pass variant per shape class: rules
+// (D, causal, smallest Sk, largest Sk, variant), first match wins, no match
+// -> variant 0.  The rows are written by the package's tuner from timings of
+// every variant on B200.
+struct VariantRule {
+  int d, causal, sk_lo, sk_hi, variant;
+};
+constexpr VariantRule kVariantRules[] = {
+#define VARIANT_RULE(d, causal, sk_lo, sk_hi, variant) {d, causal, sk_lo, sk_hi, variant},
+#include "variant_table.inc"
+#undef VARIANT_RULE
+    {0, 0, 0, 0, 0}  // end (D is never 0)
+};
+
+int select_variant(int D, int causal, int Sk) {
+  for (const VariantRule& r : kVariantRules)
+    if (r.d == D && r.causal == (causal ? 1 : 0) && Sk >= r.sk_lo && Sk <= r.sk_hi &&
+        r.variant >= 0 && r.variant < kNumVariants)
+      return r.variant;
+  return 0;
+}
+
+template <int kD>
+bool set_smem_attributes() {
+  const int bytes = static_cast<int>(fwd_smem_bytes(kD));
+  for (int v = 0; v < kNumVariants; ++v)
+    if (cudaFuncSetAttribute(fused_kernel<kD>(v), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             bytes) != cudaSuccess)
+      return false;
+  return cudaFuncSetAttribute(attn_fwd_kernel<1, kD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              bytes) == cudaSuccess;
+}
+
 attn_status device_setup(int* dev_out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ERR_CUDA;
@@ -105,14 +155,7 @@ attn_status device_setup(int* dev_out) {
     if (cudaDeviceGetAttribute(&g_dev_sms[dev], cudaDevAttrMultiProcessorCount, dev) !=
         cudaSuccess)
       return ATTN_ERR_CUDA;
-    if (cudaFuncSetAttribute(attn_fwd_kernel<0, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(fwd_smem_bytes(128))) != cudaSuccess ||
-        cudaFuncSetAttribute(attn_fwd_kernel<1, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(fwd_smem_bytes(128))) != cudaSuccess ||
-        cudaFuncSetAttribute(attn_fwd_kernel<0, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(fwd_smem_bytes(64))) != cudaSuccess ||
-        cudaFuncSetAttribute(attn_fwd_kernel<1, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(fwd_smem_bytes(64))) != cudaSuccess ||
+    if (!set_smem_attributes<128>() || !set_smem_attributes<64>() ||
         cudaFuncSetAttribute(pair::attn_fwd_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(pair_smem_bytes())) != cudaSuccess)
       return ATTN_ERR_CUDA;
@@ -232,10 +275,11 @@ bool encode_call_maps(CallMaps* m, const void* q, const void* k, const void* v, 
          encode_rows_map(&m->v, v, kv_rows, D);
 }
 
-// The fused pass over every item, then the hi+lo pass over the items it
-// listed.
+// The fused pass over every item (in the given variant), then the hi+lo pass
+// over the items it listed.
 template <int kD>
-attn_status launch_passes_d(const CallMaps& m, const FwdParams& p, int dev, cudaStream_t cs) {
+attn_status launch_passes_d(const CallMaps& m, const FwdParams& p, int variant, int dev,
+                            cudaStream_t cs) {
   const int sms = g_dev_sms[dev];
   // the pair kernel takes D = 128, Sq == Sk and whole 128-row blocks only
   if (kPairFusedPass && kD == 128 && p.S == p.Sk && p.s_tail == kBlockM) {
@@ -243,8 +287,8 @@ attn_status launch_passes_d(const CallMaps& m, const FwdParams& p, int dev, cuda
     pair::attn_fwd_pair_kernel<<<2 * pairs, pair::kThreads, pair_smem_bytes(), cs>>>(
         m.q, m.k_half, m.v, p);
   } else {
-    attn_fwd_kernel<0, kD><<<p.n_items < sms ? p.n_items : sms, kThreads, fwd_smem_bytes(kD),
-                             cs>>>(m.q, m.k, m.v, p);
+    fused_kernel<kD>(variant)<<<p.n_items < sms ? p.n_items : sms, kThreads, fwd_smem_bytes(kD),
+                                cs>>>(m.q, m.k, m.v, p);
   }
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
   attn_fwd_kernel<1, kD><<<sms, kThreads, fwd_smem_bytes(kD), cs>>>(m.q, m.k, m.v, p);
@@ -252,9 +296,10 @@ attn_status launch_passes_d(const CallMaps& m, const FwdParams& p, int dev, cuda
   return ATTN_OK;
 }
 
-attn_status launch_passes(const CallMaps& m, const FwdParams& p, int D, int dev,
+attn_status launch_passes(const CallMaps& m, const FwdParams& p, int D, int variant, int dev,
                           cudaStream_t cs) {
-  return D == 64 ? launch_passes_d<64>(m, p, dev, cs) : launch_passes_d<128>(m, p, dev, cs);
+  return D == 64 ? launch_passes_d<64>(m, p, variant, dev, cs)
+                 : launch_passes_d<128>(m, p, variant, dev, cs);
 }
 
 }  // namespace
@@ -289,11 +334,30 @@ uint64_t attn_set_wait_timeout_ns(uint64_t ns) {
   return g_timeout_ns.exchange(ns);
 }
 
-attn_status attn_fwd_qk(const void* q, const void* k, const void* v, void* o, float* lse, int B,
-                        int Hq, int Hkv, int Sq, int Sk, int D, int causal, void* stream) {
+int attn_variant_count(void) { return kNumVariants; }
+
+const char* attn_variant_name(int variant) {
+  static char names[kNumVariants][48];
+  static std::once_flag once;
+  std::call_once(once, [] {
+    for (int v = 0; v < kNumVariants; ++v)
+      std::snprintf(names[v], sizeof(names[v]), "fma_exp2_pairs=%d/8", kEmuChoices[v]);
+  });
+  return (variant >= 0 && variant < kNumVariants) ? names[variant] : nullptr;
+}
+
+int attn_variant_select(int B, int Hq, int Hkv, int Sq, int Sk, int D, int causal) {
+  if (validate_sizes(B, Hq, Hkv, Sq, D, Sk, causal) != ATTN_OK) return -1;
+  return select_variant(D, causal, Sk);
+}
+
+attn_status attn_fwd_variant(const void* q, const void* k, const void* v, void* o, float* lse,
+                             int B, int Hq, int Hkv, int Sq, int Sk, int D, int causal,
+                             int variant, void* stream) {
   if (!q || !k || !v || !o || !lse) return ATTN_ERR_NULL;
   attn_status st = validate_sizes(B, Hq, Hkv, Sq, D, Sk, causal);
   if (st != ATTN_OK) return st;
+  if (variant < 0 || variant >= kNumVariants) return ATTN_ERR_UNSUPPORTED;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
       (reinterpret_cast<uintptr_t>(lse) & 3u) != 0)
     return ATTN_ERR_ALIGN;
@@ -309,7 +373,13 @@ attn_status attn_fwd_qk(const void* q, const void* k, const void* v, void* o, fl
   if (!p.redo) return ATTN_ERR_CUDA;
   p.redo_capacity = kRedoCapacity;
 
-  return launch_passes(maps, p, D, dev, cs);
+  return launch_passes(maps, p, D, variant, dev, cs);
+}
+
+attn_status attn_fwd_qk(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                        int Hq, int Hkv, int Sq, int Sk, int D, int causal, void* stream) {
+  return attn_fwd_variant(q, k, v, o, lse, B, Hq, Hkv, Sq, Sk, D, causal,
+                          select_variant(D, causal, Sk), stream);
 }
 
 attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
@@ -541,5 +611,5 @@ extern "C" attn_status attn_fwd_noalloc(const void* q, const void* k, const void
   // the shared array keeps the previous call's header: start from an empty list
   if (cudaMemsetAsync(scratch, 0, kRedoHeaderWords * sizeof(unsigned int), cs) != cudaSuccess)
     return ATTN_ERR_CUDA;
-  return launch_passes(maps, p, D, dev, cs);
+  return launch_passes(maps, p, D, select_variant(D, causal, S), dev, cs);
 }

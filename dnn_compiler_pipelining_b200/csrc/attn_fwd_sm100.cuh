@@ -65,10 +65,14 @@ constexpr uint32_t kTileBytes = kBlockM * kHeadDim * 2;  // 32 KiB fp16 tile
 constexpr uint32_t kPanelBytes = kTileBytes / 2;         // one 64-column swizzle panel
 constexpr float kRescaleLog2 = 8.0f;
 // Of every 8 column pairs, how many take 2^x from the FMA-pipe polynomial
-// instead of the MUFU unit.  Measured on B200 (B=64, S=8192 causal): 0, 2,
-// 3, 4 pairs gave 1000, 933, 899, 861 TFLOP/s, so the MUFU unit is not this
-// kernel's limit and the polynomial stays off.
-constexpr int kEmuPairs = 0;
+// instead of the MUFU unit: the kernel's kEmu template argument, one of
+// kEmuChoices.  Which one runs for a call is a per-shape-class table measured
+// on B200.  There no class gained from the polynomial: at D = 128, S = 8192
+// causal, 0..4 pairs gave 1008, 971, 946, 911, 884 TFLOP/s, and at D = 64
+// (half the tensor work per exponential) 1 pair tied with 0 and more lost, so
+// the softmax is bound by its latency chain, not by MUFU throughput.
+constexpr int kEmuChoices[] = {0, 1, 2, 3, 4};
+constexpr int kNumVariants = sizeof(kEmuChoices) / sizeof(kEmuChoices[0]);
 constexpr float kRedoThreshold = 3.98f;
 constexpr float kLn2 = 0.69314718055994531f;
 
@@ -272,10 +276,13 @@ __device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint3
 
 // kMode 0: the fused pass over every item; kMode 1: the redo pass over the
 // listed items with hi + lo probabilities.  kD: the head dimension, 64 or 128.
-template <int kMode, int kD = 128>
+// kEmu: FMA-pipe exponentials per 8 column pairs in the fused pass (the redo
+// pass takes every exponential from the MUFU unit and is built with 0).
+template <int kMode, int kD = 128, int kEmu = 0>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+  static_assert(kEmu >= 0 && kEmu <= 8 && (kMode == 0 || kEmu == 0), "kEmu: 0..8, fused pass");
   constexpr uint32_t kTile = tile_bytes<kD>();
   constexpr int kPanels = kD / 64;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -638,8 +645,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           float lp[4] = {0.f, 0.f, 0.f, 0.f};
           if constexpr (!hilo) {
             // P rounded to fp16; l sums exactly the rounded values.  In every
-            // 16 columns, kEmuPairs pairs take 2^x from the FMA-pipe
-            // polynomial and the rest from the MUFU unit.
+            // 16 columns, kEmu pairs take 2^x from the FMA-pipe polynomial
+            // and the rest from the MUFU unit.
             const float2 sc2 = make_float2(sc, sc);
             const float2 nm2 = make_float2(neg_m, neg_m);
 #pragma unroll
@@ -651,7 +658,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                               __uint_as_float(u[c * 16 + 2 * i + 1]));
                 const float2 x2 = __ffma2_rn(s2, sc2, nm2);
                 float2 p2;
-                if (i < kEmuPairs) {
+                if (i < kEmu) {
                   p2 = exp2_poly2(x2);
                 } else {
                   p2.x = ex2_approx(x2.x);

@@ -98,6 +98,42 @@ attn_status attn_fwd_qk(const void* q, const void* k, const void* v, void* o, fl
                         void* stream);
 
 /*
+ * Fused-pass variants and their measured selection.  The pages' central idea
+ * is that the best tiling / pipeline choice of an attention kernel is found by
+ * profiling candidates on the target GPU (PipeThreader pages, sections 核心方法
+ * and 设计取舍: a joint tile + pipeline search whose greedy choices are checked
+ * by profiling); this library keeps that idea as a small build-time table.  The fused pass is compiled in
+ * attn_variant_count() variants that differ in how many of every 16
+ * exponentials of the softmax are evaluated by an FMA-pipe polynomial instead
+ * of the MUFU unit (variant i: name "fma_exp2_pairs=N/8", N pairs of 8; all
+ * variants compute the same probabilities to within the polynomial's relative
+ * error 8e-5, well inside fp16 rounding of P).  The package's tuner
+ * (python -m dnn_compiler_pipelining_b200.tune) times every variant per
+ * shape class on a B200 and writes the table compiled into the library;
+ * attn_fwd, attn_fwd_qk, attn_fwd_host and attn_fwd_noalloc run the variant
+ * the table picks.  The redo pass is the same for every variant.
+ *
+ * attn_variant_count -- number of compiled fused-pass variants (>= 1).
+ * attn_variant_name  -- static, human-readable name of a variant; NULL when
+ *                       `variant` is out of range.
+ * attn_variant_select -- the variant the table picks for these sizes, or -1
+ *                       when attn_fwd_qk would reject them (ATTN_ERR_SHAPE or
+ *                       ATTN_ERR_UNSUPPORTED).  Pure host code: no device is
+ *                       touched.
+ * attn_fwd_variant   -- attn_fwd_qk running the given fused-pass variant
+ *                       (0 <= variant < attn_variant_count(), else
+ *                       ATTN_ERR_UNSUPPORTED, checked after the sizes); for
+ *                       the tuner and tests.  Arguments, layouts and errors
+ *                       otherwise as attn_fwd_qk.
+ */
+int attn_variant_count(void);
+const char* attn_variant_name(int variant);
+int attn_variant_select(int B, int Hq, int Hkv, int Sq, int Sk, int D, int causal);
+attn_status attn_fwd_variant(const void* q, const void* k, const void* v, void* o, float* lse,
+                             int B, int Hq, int Hkv, int Sq, int Sk, int D, int causal,
+                             int variant, void* stream);
+
+/*
  * attn_fwd_host_workspace_bytes -- size in bytes of the device workspace that
  * attn_fwd_host needs for these sizes (Q, K, V, O and LSE, each rounded up to
  * 256 bytes).  Returns 0 for invalid sizes.

@@ -198,6 +198,34 @@ def test_deterministic():
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
 
 
+def test_concurrent_streams():
+    """Calls on two streams run at the same time, each with its own redo list:
+    large-V inputs (every item listed for the redo pass) on one stream and
+    N(0,1) inputs on the other give the same bytes as the same calls made one
+    after another on the default stream."""
+    B, Hq, Hkv, S, D = 2, 8, 2, 640, 128
+    qa, ka, _ = make_qkv(B, Hq, Hkv, S, D, seed=71, device="cuda")
+    va = _large_v(B, Hkv, S, D, seed=73)
+    qb, kb, vb = make_qkv(B, Hq, Hkv, S, D, seed=79, device="cuda")
+    ref_a = parity.run_gpu(qa, ka, va, True)
+    ref_b = parity.run_gpu(qb, kb, vb, False)
+    s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
+    torch.cuda.synchronize()
+    outs = []
+    for _ in range(3):
+        with torch.cuda.stream(s1):
+            oa, la = attn.attn_fwd(qa, ka, va, True, stream=s1)
+        with torch.cuda.stream(s2):
+            ob, lb = attn.attn_fwd(qb, kb, vb, False, stream=s2)
+        outs.append((oa, la, ob, lb))
+    torch.cuda.synchronize()
+    st, site = attn.device_status()
+    assert st == attn.ATTN_OK, "device status %d at site %#x" % (st, site)
+    for oa, la, ob, lb in outs:
+        assert torch.equal(oa, ref_a[0]) and torch.equal(la, ref_a[1])
+        assert torch.equal(ob, ref_b[0]) and torch.equal(lb, ref_b[1])
+
+
 def test_zero_query_prefix_mean():
     """Q = 0: O_i = mean of V_0..V_i (causal), LSE_i = ln(i+1)."""
     B, Hq, Hkv, S, D = 1, 4, 2, 512, 128
@@ -310,3 +338,52 @@ def test_fma_pipe_exp2_error_bound():
     lo = attn.selftest_exp2(torch.tensor([-125.3, -125.9, -126.0, -127.0, -200.0, -1e30,
                                           float("-inf")], device="cuda"))
     assert torch.all(lo >= 0) and torch.all(lo < 2.0 ** -124), lo
+
+
+# Every fused-pass variant (0..4 of every 8 exponential pairs from the FMA-pipe
+# polynomial) through attn_fwd_variant, against the oracle: both head dims, a
+# ragged tail, logits of standard deviation 1 and 16.
+VARIANT_CASES = [(2, 4, 2, 383, 128, 1.0), (1, 8, 2, 512, 128, 4.0), (2, 4, 2, 329, 64, 1.0),
+                 (1, 4, 2, 640, 64, 4.0)]
+
+
+def _variant_check(q, k, v, causal, variant, what):
+    o = torch.full_like(q, float("nan"))
+    lse = torch.full(q.shape[:3], float("nan"), dtype=torch.float32, device=q.device)
+    attn.attn_fwd_variant(q, k, v, causal, variant, o=o, lse=lse)
+    st, site = attn.device_status()
+    assert st == attn.ATTN_OK, "device status %d at site %#x" % (st, site)
+    o_ref, lse_ref = parity.oracle.attention(q.cpu().double().numpy(), k.cpu().double().numpy(),
+                                             v.cpu().double().numpy(), causal)
+    parity.assert_close(o.cpu().double().numpy(), o_ref, lse.cpu().double().numpy(), lse_ref,
+                        what)
+
+
+@pytest.mark.parametrize("variant", range(5))
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("B,Hq,Hkv,S,D,qk_std", VARIANT_CASES)
+def test_variant_full(B, Hq, Hkv, S, D, qk_std, causal, variant):
+    assert attn.variant_count() == 5
+    q, k, v = make_qkv(B, Hq, Hkv, S, D, seed=41, qk_std=qk_std, device="cuda")
+    _variant_check(q, k, v, causal, variant, "%s B%d Hq%d S%d D%d std%g causal=%d" % (
+        attn.variant_name(variant), B, Hq, S, D, qk_std, causal))
+
+
+@pytest.mark.parametrize("variant", [2, 4])
+def test_variant_large_outputs(variant):
+    """Large V: every item goes through the redo pass after an emulating fused pass."""
+    q, k, _ = make_qkv(1, 8, 2, 384, 128, seed=43, device="cuda")
+    v = _large_v(1, 2, 384, 128, seed=47)
+    _variant_check(q, k, v, True, variant, "large V, %s" % attn.variant_name(variant))
+
+
+def test_variant_default_is_table_choice():
+    """attn_fwd runs the variant attn_variant_select names: same bytes."""
+    for D in (64, 128):
+        q, k, v = make_qkv(1, 8, 2, 1024, D, seed=53, device="cuda")
+        var = attn.variant_select(1, 8, 2, 1024, 1024, D, True)
+        assert 0 <= var < attn.variant_count()
+        o1, l1 = parity.run_gpu(q, k, v, True)
+        o2, l2 = attn.attn_fwd_variant(q, k, v, True, var)
+        torch.cuda.synchronize()
+        assert torch.equal(o1, o2) and torch.equal(l1, l2)
