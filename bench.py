@@ -411,6 +411,87 @@ def run_gpu(args, w, name):
         dist.destroy_process_group()
 
 
+# --------------------------------------------------------------------------- decoder layer
+def layer_flops(B, S, hidden, Hq, Hkv, D, inter):
+    """GEMM FLOPs of one decoder layer plus its causal attention."""
+    T = B * S
+    gemm = 2.0 * T * hidden * ((Hq + 2 * Hkv) * D + Hq * D + 2 * inter + inter)
+    return gemm + attn_flops(B, Hq, S, D, True)
+
+
+def run_layer(args):
+    """One LLaMA3 decoder layer (attn_decoder_layer_fwd) per step, 1 GPU; prints
+    its own JSON line (not the attention headline)."""
+    import torch
+    from dnn_compiler_pipelining_b200 import attn
+    from dnn_compiler_pipelining_b200.inputs import DECODER_MODELS, make_decoder_inputs, make_qkv
+
+    m = DECODER_MODELS[args.layer]
+    B, S = args.layer_batch, args.layer_seq
+    hidden, Hq, Hkv, D, inter = m["hidden"], m["Hq"], m["Hkv"], m["D"], m["inter"]
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    attn.load()
+    x, w = make_decoder_inputs(B, S, hidden, Hq, Hkv, D, inter, seed=0, device=dev)
+    y = torch.empty_like(x)
+    ws = torch.empty(attn.decoder_layer_workspace_bytes(B, S, hidden, Hq, Hkv, D, inter),
+                     dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        attn.decoder_layer_fwd(x, w, Hq, Hkv, D, y=y, workspace=ws, stream=stream)
+
+    def timed(fn, n):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(dev)
+        e0.record(stream)
+        for _ in range(n):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        return e0.elapsed_time(e1) / n
+
+    for _ in range(args.warmup):
+        step()
+    with ClockSampler(0) as clk:
+        ms = timed(step, args.steps)
+    clocks = clk.summary()
+    st, site = attn.device_status()
+    if st != attn.ATTN_OK:
+        raise RuntimeError("device status %d at site %#x" % (st, site))
+    # the attention alone on the same shape, for the split of the step
+    q, k, v = make_qkv(B, Hq, Hkv, S, D, seed=1, device=dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, Hq, S), dtype=torch.float32, device=dev)
+    for _ in range(args.warmup):
+        attn.attn_fwd(q, k, v, True, o=o, lse=lse, stream=stream)
+    attn_ms = timed(lambda: attn.attn_fwd(q, k, v, True, o=o, lse=lse, stream=stream), args.steps)
+    flops = layer_flops(B, S, hidden, Hq, Hkv, D, inter)
+    peaks, src = load_peaks()
+    peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    value = flops / (ms * 1e-3) / 1e12
+    line = {
+        "metric": "decoder layer fwd TFLOP/s (fp16, LLaMA3 single-layer proxy)",
+        "value": value, "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f16", "data": "synthetic (random weights)",
+        "config": {"workload": "%s-layer-s%d-b%d" % (args.layer, S, B), "B": B, "S": S,
+                   "hidden": hidden, "Hq": Hq, "Hkv": Hkv, "D": D, "inter": inter,
+                   "causal": True, "l2": "activations and weights larger than L2"},
+        "roofline": {"bound": "tensor", "achieved": value, "peak": peak, "unit": "TFLOP/s",
+                     "frac": value / peak, "traffic": None,
+                     "peak_source": "%s bf16 dense GEMM, sustained" % src,
+                     "algorithmic_flops_per_step": flops},
+        "split": {"attention_ms": attn_ms, "rest_ms": ms - attn_ms,
+                  "attention_flops": attn_flops(B, Hq, S, D, True)},
+        "clocks": clocks,
+        # per step: rope table, 2 RMSNorm, RoPE split, the 2 attention passes,
+        # head merge, SwiGLU; plus 4 cuBLAS GEMM calls
+        "gpu_launches": 8 * args.steps, "library_gemm_calls": 4 * args.steps,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main(argv=None):
     from dnn_compiler_pipelining_b200.inputs import WORKLOADS
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
@@ -424,11 +505,19 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-seconds", type=float, default=8.0)
+    ap.add_argument("--layer", choices=["llama3-8b", "llama3-70b"], default=None,
+                    help="time the decoder-layer proxy instead of the attention headline")
+    ap.add_argument("--layer-batch", type=int, default=1)
+    ap.add_argument("--layer-seq", type=int, default=8192)
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "ours":
         ap.error("--warmup must be at least 3")
     w = WORKLOADS[args.workload]
-    if args.impl == "reference":
+    if args.layer is not None:
+        if args.impl != "ours":
+            ap.error("--layer times this library only")
+        run_layer(args)
+    elif args.impl == "reference":
         run_reference(args, w, args.workload)
     else:
         run_gpu(args, w, args.workload)

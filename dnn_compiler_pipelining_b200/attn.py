@@ -53,6 +53,10 @@ def load() -> ctypes.CDLL:
     lib.attn_variant_name.restype = ctypes.c_char_p
     lib.attn_variant_select.argtypes = [i, i, i, i, i, i, i]
     lib.attn_variant_select.restype = i
+    lib.attn_decoder_layer_workspace_bytes.argtypes = [i] * 7
+    lib.attn_decoder_layer_workspace_bytes.restype = sz
+    lib.attn_decoder_layer_fwd.argtypes = [vp] * 8 + [i] * 7 + [ctypes.c_float] * 2 + [vp, sz, vp]
+    lib.attn_decoder_layer_fwd.restype = i
     lib.attn_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, vp]
     lib.attn_fwd_noalloc.restype = i
     lib.attn_fwd_host.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, vp, sz, vp]
@@ -192,6 +196,47 @@ def attn_fwd_noalloc_raw(q_ptr: int, k_ptr: int, v_ptr: int, o_ptr: int, lse_ptr
     device."""
     return int(load().attn_fwd_noalloc(q_ptr, k_ptr, v_ptr, o_ptr, lse_ptr, B, Hq, Hkv, S, D,
                                        int(bool(causal)), stream_ptr))
+
+
+DECODER_WEIGHTS = ("w_attn_norm", "w_qkv", "w_o", "w_mlp_norm", "w_gate_up", "w_down")
+
+
+def decoder_layer_workspace_bytes(B: int, S: int, hidden: int, Hq: int, Hkv: int, D: int,
+                                  inter: int) -> int:
+    return int(load().attn_decoder_layer_workspace_bytes(B, S, hidden, Hq, Hkv, D, inter))
+
+
+def decoder_layer_fwd(x: torch.Tensor, weights: dict, Hq: int, Hkv: int, D: int,
+                      eps: float = 1e-5, rope_theta: float = 500000.0,
+                      y: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+                      stream=None) -> torch.Tensor:
+    """One LLaMA3 decoder layer (include/decoder_layer.h) on CUDA fp16 tensors.
+
+    x: [B, S, hidden]; weights: the six tensors named in DECODER_WEIGHTS, laid
+    out as the C ABI states.  y (default: new) may be x itself.  workspace:
+    a CUDA uint8 tensor of at least decoder_layer_workspace_bytes(...) bytes
+    (default: allocated here).  Asynchronous on ``stream``."""
+    lib = load()
+    _check_dev(x, "x", torch.float16)
+    B, S, hidden = x.shape
+    inter = weights["w_down"].shape[1]
+    for name in DECODER_WEIGHTS:
+        _check_dev(weights[name], name, torch.float16)
+    if y is None:
+        y = torch.empty_like(x)
+    _check_dev(y, "y", torch.float16)
+    need = decoder_layer_workspace_bytes(B, S, hidden, Hq, Hkv, D, inter)
+    if need == 0:
+        raise AttnError(2, "attn_decoder_layer_workspace_bytes")
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    st = lib.attn_decoder_layer_fwd(
+        x.data_ptr(), *[weights[n].data_ptr() for n in DECODER_WEIGHTS], y.data_ptr(), B, S,
+        hidden, Hq, Hkv, D, inter, float(eps), float(rope_theta), workspace.data_ptr(),
+        workspace.numel() * workspace.element_size(), _stream_ptr(stream))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_decoder_layer_fwd")
+    return y
 
 
 def host_workspace_bytes(B: int, Hq: int, Hkv: int, S: int, D: int) -> int:

@@ -13,10 +13,10 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libattn_b200.so")
-SOURCES = [os.path.join(CSRC, "attn_api.cu")]
+SOURCES = [os.path.join(CSRC, "attn_api.cu"), os.path.join(CSRC, "decoder_api.cu")]
 DEPS = SOURCES + [os.path.join(CSRC, f) for f in os.listdir(CSRC)
                   if f.endswith(".cuh") or f.endswith(".inc")] + \
-    [os.path.join(INCLUDE, "attn.h")]
+    [os.path.join(INCLUDE, f) for f in os.listdir(INCLUDE) if f.endswith(".h")]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = [
@@ -25,6 +25,7 @@ FLAGS = [
     "-Xcompiler", "-fPIC", "-shared",
     "-I", INCLUDE, "-I", CSRC,
 ]
+LIBS = ["-lcublas"]
 
 
 def build(force: bool = False, verbose: bool = False) -> str:
@@ -32,7 +33,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
     if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= newest:
         return LIB
     tmp = LIB + ".tmp.%d" % os.getpid()
-    cmd = [NVCC] + FLAGS + (["-Xptxas", "-v"] if verbose else []) + ["-o", tmp] + SOURCES
+    cmd = [NVCC] + FLAGS + (["-Xptxas", "-v"] if verbose else []) + ["-o", tmp] + SOURCES + LIBS
     subprocess.check_call(cmd)
     os.replace(tmp, LIB)
     return LIB

@@ -25,7 +25,7 @@ import torch
 _CHUNK_ELEMS = 1 << 26  # fp32 temporaries of at most 256 MiB
 
 
-def _normal_fp16(shape, seed: int, std: float, device) -> torch.Tensor:
+def _normal_fp16(shape, seed: int, std: float, device, mean: float = 0.0) -> torch.Tensor:
     gen = torch.Generator(device=device)
     gen.manual_seed(int(seed))
     out = torch.empty(shape, dtype=torch.float16, device=device)
@@ -37,6 +37,8 @@ def _normal_fp16(shape, seed: int, std: float, device) -> torch.Tensor:
         x = torch.randn(m, generator=gen, dtype=torch.float32, device=device)
         if std != 1.0:
             x.mul_(std)
+        if mean != 0.0:
+            x.add_(mean)
         flat[start:start + m].copy_(x)
     return out
 
@@ -74,3 +76,33 @@ def sweep_points():
                     pts.append(dict(B=B, Hq=Hq, Hkv=8, S=S, D=128, causal=causal))
     return pts
 
+
+
+# Decoder-layer proxy (the pages' second workload: an FP16 single LLaMA3-8B /
+# 70B decoder layer, papers.lqhl.me "PipeThreader-OSDI25", paper Sec. 6.3 /
+# Fig. 13): model dimensions of the two LLaMA3 sizes.
+DECODER_MODELS = {
+    "llama3-8b": dict(hidden=4096, Hq=32, Hkv=8, D=128, inter=14336),
+    "llama3-70b": dict(hidden=8192, Hq=64, Hkv=8, D=128, inter=28672),
+}
+
+
+def make_decoder_inputs(B: int, S: int, hidden: int, Hq: int, Hkv: int, D: int, inter: int,
+                        seed: int = 0, device="cpu"):
+    """Synthetic activations and weights of one decoder layer, fp16 on ``device``.
+
+    x ~ N(0, 1) [B, S, hidden]; each projection W [out, in] ~ N(0, 1/in), so
+    every product keeps unit scale; the two RMSNorm weights ~ N(1, 0.1^2).
+    Tensor k of (x, w_attn_norm, w_qkv, w_o, w_mlp_norm, w_gate_up, w_down)
+    uses seed + k.  Returns (x, weights dict keyed as the C ABI names them).
+    """
+    x = _normal_fp16((B, S, hidden), seed, 1.0, device)
+    w = {
+        "w_attn_norm": _normal_fp16((hidden,), seed + 1, 0.1, device, mean=1.0),
+        "w_qkv": _normal_fp16(((Hq + 2 * Hkv) * D, hidden), seed + 2, hidden ** -0.5, device),
+        "w_o": _normal_fp16((hidden, Hq * D), seed + 3, (Hq * D) ** -0.5, device),
+        "w_mlp_norm": _normal_fp16((hidden,), seed + 4, 0.1, device, mean=1.0),
+        "w_gate_up": _normal_fp16((2 * inter, hidden), seed + 5, hidden ** -0.5, device),
+        "w_down": _normal_fp16((hidden, inter), seed + 6, inter ** -0.5, device),
+    }
+    return x, w

@@ -1,4 +1,4 @@
-"""The C-ABI library on the CPU: it loads, exports every symbol include/attn.h
+"""The C-ABI library on the CPU: it loads, exports every symbol include/*.h
 declares, and rejects bad arguments before touching a GPU.  No compute call
 runs here (this machine has no GPU)."""
 import ctypes
@@ -12,7 +12,6 @@ from dnn_compiler_pipelining_b200 import attn
 from dnn_compiler_pipelining_b200.build import build
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-HEADER = os.path.join(ROOT, "include", "attn.h")
 
 OK, NULL, SHAPE, ALIGN, UNSUP, CUDA, TIMEOUT, WORKSPACE = range(8)
 
@@ -24,7 +23,8 @@ def lib():
 
 
 def declared_functions():
-    text = open(HEADER).read()
+    text = "".join(open(os.path.join(ROOT, "include", f)).read()
+                   for f in sorted(os.listdir(os.path.join(ROOT, "include"))) if f.endswith(".h"))
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
     return sorted(set(re.findall(r"\b(attn_[a-z0-9_]+)\s*\(", text)))
 
