@@ -2,14 +2,20 @@
 the C ABI) against the fp64 oracle, which rounds to fp16 at the same points
 where the layer stores a tensor.  Needs a B200.
 
-Tolerance, from the arithmetic: both sides round the same steps to fp16, so
-they differ by fp32-vs-fp64 arithmetic inside a step (relative ~1e-6), by the
-attention kernel's own error (max 2e-3 on O, which the output projection
-averages down), and by the occasional one-step rounding flip of an
-intermediate, which reaches y through the residual h = x + ... at most one
-fp16 step of |h| ~ |y|, plus y's own rounding.  Bound per element:
-|y_gpu - y_ref| <= 2e-3 + 4 * ulp16(|y_ref|), where ulp16(v) is the fp16
-spacing at v; and the mean error <= 5e-4."""
+Tolerance, from the arithmetic.  Both sides round the same steps to fp16, so
+they differ only by:
+  * fp32-vs-fp64 arithmetic inside a step (relative ~1e-6);
+  * the attention kernel's own error (up to 2e-3 on O);
+  * one-step fp16 rounding flips of intermediates, which those differences
+    trigger.
+A difference in an intermediate reaches y in two ways:
+  * through a projection sum, whose terms each carry up to 2^-11 relative
+    error, giving an absolute error that scales with the RMS of the output
+    row, not with the element itself;
+  * through the residual h = x + ..., at most a fp16 step or two of |y|.
+Bound per element: |y_gpu - y_ref| <= 4 ulp16(|y_ref|) + 8 * 2^-11 * rms(y_ref
+row), where ulp16(v) is the fp16 spacing at v.  On average the difference is
+at most one fp16 step: mean |y_gpu - y_ref| <= mean ulp16(|y_ref|)."""
 import numpy as np
 import pytest
 import torch
@@ -54,11 +60,14 @@ def _check(x, w, y, Hq, Hkv, D, what):
     got = y.cpu().double().numpy()
     assert np.all(np.isfinite(got)), what + ": non-finite output"
     err = np.abs(got - ref)
-    bound = 2e-3 + 4 * ulp16(ref)
-    worst = np.unravel_index(np.argmax(err - bound), err.shape)
+    rms = np.sqrt(np.mean(ref * ref, axis=-1, keepdims=True))
+    bound = 4 * ulp16(ref) + 8 * 2.0 ** -11 * rms
+    worst = np.unravel_index(np.argmax(err / bound), err.shape)
     assert np.all(err <= bound), "%s: err %.3e > bound %.3e at %s (ref %.4f)" % (
         what, err[worst], bound[worst], worst, ref[worst])
-    assert err.mean() <= 5e-4, "%s: mean err %.3e" % (what, err.mean())
+    assert err.mean() <= ulp16(ref).mean(), "%s: mean err %.3e > mean fp16 step %.3e" % (
+        what, err.mean(), ulp16(ref).mean())
+    print("%s: max err / bound %.2f, mean err %.2e" % (what, (err / bound).max(), err.mean()))
 
 
 # (B, S, hidden, Hq, Hkv, D, inter): several tiles, ragged S, both head dims
