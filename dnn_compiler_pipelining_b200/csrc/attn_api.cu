@@ -1,7 +1,8 @@
 // attn_api.cu -- C ABI of libattn_b200.so (declared in include/attn.h):
 // argument validation, TMA tensor-map encoding, kernel launch, the
 // per-device status word, the host-buffer entry point and the bounded-wait
-// self-test.  Nothing here allocates device memory.
+// self-test.  The only device memory it allocates is the redo list of each
+// (device, stream) pair, once, on first use.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
