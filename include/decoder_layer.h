@@ -75,8 +75,10 @@ size_t attn_decoder_layer_workspace_bytes(int B, int S, int hidden, int Hq, int 
  * Returns ATTN_OK once everything is enqueued; ATTN_ERR_NULL, ATTN_ERR_SHAPE
  * (sizes, eps, theta), ATTN_ERR_UNSUPPORTED (D), ATTN_ERR_ALIGN,
  * ATTN_ERR_WORKSPACE before launching anything; ATTN_ERR_CUDA when a launch or
- * a cuBLAS call fails; the attention's status otherwise.  A timed-out wait in
- * the attention is reported by attn_device_status().
+ * a cuBLAS call fails; the attention's status otherwise.  After a failure past
+ * validation, earlier steps may already be enqueued: y and the workspace are
+ * then undefined.  A timed-out wait in the attention is reported by
+ * attn_device_status().
  */
 attn_status attn_decoder_layer_fwd(const void* x, const void* w_attn_norm, const void* w_qkv,
                                    const void* w_o, const void* w_mlp_norm, const void* w_gate_up,
