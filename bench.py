@@ -447,6 +447,39 @@ def layer_flops(B, S, hidden, Hq, Hkv, D, inter):
     return gemm + attn_flops(B, Hq, S, D, True)
 
 
+def blas_threads():
+    """Threads numpy's BLAS runs the oracle's matrix products on."""
+    try:
+        from threadpoolctl import threadpool_info
+        n = [p["num_threads"] for p in threadpool_info() if p.get("user_api") == "blas"]
+        return max(n) if n else os.cpu_count()
+    except ImportError:
+        return os.cpu_count()
+
+
+def layer_oracle_sample(m, seconds: float, S: int = 128, seed: int = 0):
+    """Time the fp64 decoder-layer oracle on whole B=1 sequences of S tokens at
+    the model's dimensions until about `seconds` of CPU work.  Returns (flops
+    done, seconds, tokens)."""
+    from oracle import decoder as oracle_decoder
+    from dnn_compiler_pipelining_b200.inputs import make_decoder_inputs
+
+    hidden, Hq, Hkv, D, inter = m["hidden"], m["Hq"], m["Hkv"], m["D"], m["inter"]
+    x, w = make_decoder_inputs(1, S, hidden, Hq, Hkv, D, inter, seed=seed, device="cpu")
+    xd = x.double().numpy()
+    wd = {k: v.double().numpy() for k, v in w.items()}
+    flops, tokens = 0.0, 0
+    t0 = time.perf_counter()
+    while True:
+        oracle_decoder.decoder_layer(xd, Hq=Hq, Hkv=Hkv, D=D, eps=1e-5, theta=500000.0, **wd)
+        flops += layer_flops(1, S, hidden, Hq, Hkv, D, inter)
+        tokens += S
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            break
+    return flops, el, tokens
+
+
 def run_layer(args):
     """One LLaMA3 decoder layer (attn_decoder_layer_fwd) per step, 1 GPU; prints
     its own JSON line (not the attention headline)."""
@@ -517,6 +550,12 @@ def run_layer(args):
         # head merge, SwiGLU; plus 4 cuBLAS GEMM calls
         "gpu_launches": 8 * args.steps, "library_gemm_calls": 4 * args.steps,
     }
+    if not args.no_cpu_baseline:
+        f, t, n = layer_oracle_sample(m, args.cpu_seconds)
+        line["cpu_baseline"] = {
+            "value": f / t / 1e12, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": "%d tokens in whole 128-token sequences (B=1) at the model's dimensions, "
+                      "%.1f s of fp64 oracle work (numpy BLAS threads)" % (n, t)}
     print(json.dumps(line), flush=True)
 
 
