@@ -24,8 +24,8 @@ def lib():
     return attn.load()
 
 
-def table_rules():
-    text = re.sub(r"//[^\n]*", "", open(TABLE).read())
+def table_rules(path=TABLE):
+    text = re.sub(r"//[^\n]*", "", open(path).read())
     return [tuple(int(x) for x in m.groups()) for m in re.finditer(
         r"VARIANT_RULE\(\s*(-?\d+)\s*,\s*(-?\d+)\s*,\s*(-?\d+)\s*,\s*(-?\d+)\s*,\s*(-?\d+)\s*\)",
         text)]
@@ -120,3 +120,41 @@ def test_tuner_rules_cover_all_sizes():
     # boundaries sit at geometric midpoints: 724 (sqrt(512 * 1024) = 724.08) -> 512's rule
     assert rules[0] == (1, int(math.sqrt(512 * 1024)), 0)
     assert tune.rules_for([(512, 3)]) == [(1, 2 ** 31 - 1, 3)]
+
+
+def test_tuner_writes_a_table_the_library_format_accepts(tmp_path, monkeypatch):
+    """tune.main with the GPU timing replaced by a fake: the table it writes has
+    one rule set per (D, causal), parses with the same pattern the library's
+    macro takes, and picks a faster agreeing variant only past the margin."""
+    fake = {}
+
+    def fake_time_class(D, causal, S, reps, warmup, seed=0):
+        med = [1.0, 1.0, 1.0, 1.0, 1.0]
+        if D == 64 and causal and S >= 2048:
+            med[2] = 0.9          # 10 % faster: chosen
+        if D == 128 and not causal and S == 512:
+            med[1] = 0.99         # 1 % faster: under the margin
+        fake[(D, causal, S)] = med
+        return max(1, tune.TOKENS // S), med, [True] * 5
+
+    class Props:
+        name, multi_processor_count = "fake GPU", 148
+
+    monkeypatch.setattr(tune, "time_class", fake_time_class)
+    monkeypatch.setattr(tune.torch.cuda, "is_available", lambda: True)
+    monkeypatch.setattr(tune.torch.cuda, "get_device_properties", lambda i: Props())
+    monkeypatch.setattr(tune.attn, "variant_count", lambda: 5)
+    monkeypatch.setattr(tune.attn, "variant_name", lambda i: "v%d" % i)
+    table, report = tmp_path / "t.inc", tmp_path / "r.md"
+    tune.main(["--table", str(table), "--report", str(report)])
+    text = open(table).read()
+    rules = table_rules(str(table))
+    assert len(fake) == 20
+    assert expected_variant(rules, 64, 1, 8192) == 2 and expected_variant(rules, 64, 1, 2048) == 2
+    # 1448 is the geometric midpoint of 1024 and 2048: the 2048 rule starts just above it
+    assert expected_variant(rules, 64, 1, 1448) == 0 and expected_variant(rules, 64, 1, 1449) == 2
+    assert expected_variant(rules, 128, 0, 512) == 0
+    assert all(expected_variant(rules, d, c, s) == 0 for d in (64, 128) for c in (0, 1)
+               for s in (1, 512, 1024) if not (d == 64 and c == 1 and s >= 1449))
+    assert "VARIANT_RULE(" in text and "fake GPU" in text
+    assert "| 64 | 1 | 8192 |" in open(report).read()
