@@ -2,10 +2,11 @@
 // layer proxy around the attention forward (the PipeThreader pages' second
 // workload: an FP16 single decoder layer of LLaMA3-8B / 70B, section 实验与结果,
 // paper Sec. 6.3 / Fig. 13).  The GEMMs are library calls; the attention is
-// this library's fused kernel.  Every kernel here is bound by HBM traffic: it
-// reads and writes each element once with 16-byte vector accesses (rows are
-// multiples of 8 fp16 elements and 16-byte aligned, which the entry point
-// checks), and computes in fp32 with one rounding to fp16 per output.
+// this library's fused kernel.  Every kernel here is bound by HBM traffic: each
+// element crosses HBM once in each direction, with 16-byte vector accesses.
+// Rows are multiples of 8 fp16 elements and 16-byte aligned, which the entry
+// point checks; RMSNorm's second read of a row hits L1/L2.  Each computes in
+// fp32 with one rounding to fp16 per output.
 #pragma once
 
 #include <cuda_fp16.h>
