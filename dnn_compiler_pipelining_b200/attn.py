@@ -65,6 +65,12 @@ def load() -> ctypes.CDLL:
     lib.attn_fwd_host_workspace_bytes.restype = sz
     lib.attn_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32)]
     lib.attn_device_status.restype = i
+    lib.attn_device_status_ex.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32),
+                                          ctypes.POINTER(ctypes.c_uint64)]
+    lib.attn_device_status_ex.restype = i
+    lib.attn_noalloc_status.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32),
+                                        ctypes.POINTER(ctypes.c_uint64)]
+    lib.attn_noalloc_status.restype = i
     lib.attn_set_wait_timeout_ns.argtypes = [u64]
     lib.attn_set_wait_timeout_ns.restype = u64
     lib.attn_selftest_exp2.argtypes = [vp, vp, i, vp]
@@ -190,10 +196,9 @@ def attn_fwd_noalloc_raw(q_ptr: int, k_ptr: int, v_ptr: int, o_ptr: int, lse_ptr
     """The no-allocation C entry point with raw addresses; returns the status
     code.  For callers that cannot let the library call cudaMalloc (memory
     planned up front, their own caching allocator, or no tolerance for the
-    device synchronization an allocation may cause): its scratch is a fixed
-    array inside the library, so sizes above B*Hq*ceil(S/256) = 131072 work
-    items are rejected, and calls that overlap on the GPU must not share a
-    device."""
+    device synchronization an allocation may cause): its per-call status
+    words are a fixed array inside the library (read them with
+    noalloc_status), shared by every such call on a device."""
     return int(load().attn_fwd_noalloc(q_ptr, k_ptr, v_ptr, o_ptr, lse_ptr, B, Hq, Hkv, S, D,
                                        int(bool(causal)), stream_ptr))
 
@@ -262,10 +267,28 @@ def attn_fwd_host(q_h: torch.Tensor, k_h: torch.Tensor, v_h: torch.Tensor, o_h: 
 
 
 def device_status(stream=None):
-    """(status, site): synchronizes, reads and clears the device status word."""
+    """(status, site): synchronizes the stream, reads and clears its status block."""
     site = ctypes.c_uint32(0)
     st = load().attn_device_status(_stream_ptr(stream), ctypes.byref(site))
     return int(st), int(site.value)
+
+
+def device_status_ex(stream=None):
+    """(status, site, exact_items): as device_status, plus how many work items
+    the kernels recomputed in their exact pass since the last read."""
+    site = ctypes.c_uint32(0)
+    n = ctypes.c_uint64(0)
+    st = load().attn_device_status_ex(_stream_ptr(stream), ctypes.byref(site), ctypes.byref(n))
+    return int(st), int(site.value), int(n.value)
+
+
+def noalloc_status(stream=None):
+    """(status, site, exact_items) of the attn_fwd_noalloc calls on this device
+    since the last read; synchronizes the stream, then clears the words."""
+    site = ctypes.c_uint32(0)
+    n = ctypes.c_uint64(0)
+    st = load().attn_noalloc_status(_stream_ptr(stream), ctypes.byref(site), ctypes.byref(n))
+    return int(st), int(site.value), int(n.value)
 
 
 def set_wait_timeout_ns(ns: int) -> int:

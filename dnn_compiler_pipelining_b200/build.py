@@ -25,7 +25,7 @@ FLAGS = [
     "-Xcompiler", "-fPIC", "-shared",
     "-I", INCLUDE, "-I", CSRC,
 ]
-LIBS = ["-lcublas"]
+LIBS = []
 
 
 def build(force: bool = False, verbose: bool = False) -> str:

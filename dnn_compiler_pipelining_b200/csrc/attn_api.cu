@@ -1,8 +1,8 @@
 // attn_api.cu -- C ABI of libattn_b200.so (declared in include/attn.h):
-// argument validation, TMA tensor-map encoding, kernel launch, the
-// per-device status word, the host-buffer entry point and the bounded-wait
-// self-test.  The only device memory it allocates is the redo list of each
-// (device, stream) pair, once, on first use.
+// argument validation, TMA tensor-map encoding, kernel launch, the per-call
+// status blocks, the host-buffer entry point and the self-tests.  The only
+// device memory it allocates is one small status block per (device, stream)
+// -- per (device, host thread) for cudaStreamPerThread -- once, on first use.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
@@ -14,10 +14,12 @@
 #include <cstdio>
 #include <map>
 #include <mutex>
+#include <thread>
+#include <tuple>
 #include <utility>
 
 #include "attn.h"
-#include "attn_fwd_pair_sm100.cuh"
+#include "attn_fwd_db_sm100.cuh"
 #include "attn_fwd_sm100.cuh"
 
 namespace attn_b200 {
@@ -41,70 +43,61 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// Per-device one-time setup: architecture check and the kernel's shared
-// memory opt-in.  0 = not done, 1 = ok, 2 = unsupported device.
-std::atomic<int> g_dev_state[kMaxDevices];
-int g_dev_sms[kMaxDevices];
-int g_dev_pairs[kMaxDevices];  // 2-CTA clusters of the pair kernel resident at once
-std::mutex g_dev_mutex;
+// ---------------------------------------------------------------------------
+// fused-kernel variants: a pipeline structure x kEmu FMA-pipe exponentials
+// per 8 column pairs.  Structures: 0 two-tile ping-pong, one MMA-issuing
+// warp; 1 the same with one issuing warp per tile; 2 one tile with S
+// double-buffered in TMEM; 3 the same with two softmax warps per lane
+// quadrant.  Head dimension 256 has only the double-buffered kernel with one
+// softmax warp per quadrant (shared memory has no room for more): every
+// structure maps to it there.
+// ---------------------------------------------------------------------------
+constexpr int kEmuChoices = kEmuMax + 1;  // 0..4
+constexpr int kStructures = 4;
+constexpr int kNumVariants = kStructures * kEmuChoices;
+__host__ __device__ constexpr int variant_emu(int v) { return v % kEmuChoices; }
+__host__ __device__ constexpr int variant_structure(int v) { return v / kEmuChoices; }
 
-// Redo lists (items the fast pass hands to the hi+lo pass), one per
-// (device, stream): launches on one stream run in order, so a list is never
-// shared by launches that could overlap.
-constexpr unsigned int kRedoCapacity = 1u << 16;
-std::map<std::pair<int, cudaStream_t>, unsigned int*> g_redo_lists;
-std::mutex g_redo_mutex;
-
-size_t redo_bytes() { return (kRedoHeaderWords + kRedoCapacity) * sizeof(unsigned int); }
-
-// Returns the list for (dev, stream), allocating and zeroing it (on that
-// stream) the first time.
-unsigned int* redo_list(int dev, cudaStream_t stream) {
-  std::lock_guard<std::mutex> lock(g_redo_mutex);
-  auto key = std::make_pair(dev, stream);
-  auto it = g_redo_lists.find(key);
-  if (it != g_redo_lists.end()) return it->second;
-  void* ptr = nullptr;
-  if (cudaMalloc(&ptr, redo_bytes()) != cudaSuccess) return nullptr;
-  if (cudaMemsetAsync(ptr, 0, redo_bytes(), stream) != cudaSuccess) {
-    cudaFree(ptr);
-    return nullptr;
-  }
-  g_redo_lists[key] = static_cast<unsigned int*>(ptr);
-  return static_cast<unsigned int*>(ptr);
-}
-
-// Which kernel runs the fused pass: the single-CTA kernel (attn_fwd_kernel<0>)
-// or the CTA-pair kernel (pair::attn_fwd_pair_kernel), which computes the
-// same items and passes the same parity tests but measured slower on B200
-// (793 vs 1003 TFLOP/s at B=64, S=8192, causal).
-constexpr bool kPairFusedPass = false;
-
-// the kernel checks 1 KiB alignment of the dynamic shared memory base
-size_t fwd_smem_bytes(int D = kHeadDim) {
-  return D == 64 ? sizeof(SharedFwdT<64>) : sizeof(SharedFwdT<128>);
-}
-size_t pair_smem_bytes() { return sizeof(pair::SharedPair); }
-
-// The fused-pass kernels of one head dimension, indexed by variant
-// (kEmuChoices[variant] FMA-pipe exponentials per 8 column pairs).
 using FwdKernel = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap,
                            const FwdParams);
+struct KernelChoice {
+  FwdKernel fn;
+  size_t smem;
+  int one_tile;  // items are one 128-row tile
+  int kv_box;    // rows of a K / V tile
+};
+
+template <int kD, int kV>
+KernelChoice kernel_choice_v() {
+  constexpr int s = variant_structure(kV), e = variant_emu(kV);
+  if constexpr (kD == 256) {
+    return {&db::attn_fwd_db_kernel<256, 1, e>, sizeof(db::SharedDb<256, 1>), 1,
+            db::Cfg<256>::kBN};
+  } else if constexpr (s == 0 || s == 1) {
+    return {&attn_fwd_kernel<kD, e, s + 1>, sizeof(SharedFwdT<kD>), 0, kBlockN};
+  } else {
+    return {&db::attn_fwd_db_kernel<kD, s - 1, e>, sizeof(db::SharedDb<kD, s - 1>), 1,
+            db::Cfg<kD>::kBN};
+  }
+}
 template <int kD, int... kV>
-std::array<FwdKernel, sizeof...(kV)> fused_kernels(std::integer_sequence<int, kV...>) {
-  return {{&attn_fwd_kernel<0, kD, kEmuChoices[kV]>...}};
+std::array<KernelChoice, sizeof...(kV)> kernel_table(std::integer_sequence<int, kV...>) {
+  return {{kernel_choice_v<kD, kV>()...}};
 }
 template <int kD>
-FwdKernel fused_kernel(int variant) {
-  static const std::array<FwdKernel, kNumVariants> table =
-      fused_kernels<kD>(std::make_integer_sequence<int, kNumVariants>{});
+const KernelChoice& kernel_choice_d(int variant) {
+  static const std::array<KernelChoice, kNumVariants> table =
+      kernel_table<kD>(std::make_integer_sequence<int, kNumVariants>{});
   return table[variant];
 }
+const KernelChoice& kernel_choice(int D, int variant) {
+  return D == 64 ? kernel_choice_d<64>(variant)
+                 : D == 128 ? kernel_choice_d<128>(variant) : kernel_choice_d<256>(variant);
+}
 
-// Measured choice of fused-pass variant per shape class: rules
-// (D, causal, smallest Sk, largest Sk, variant), first match wins, no match
-// -> variant 0.  The rows are written by the package's tuner from timings of
-// every variant on B200.
+// Measured choice of variant per shape class: rules (D, causal, smallest Sk,
+// largest Sk, variant), first match wins, no match -> variant 0.  The rows
+// are written by the package's tuner from timings of every variant on B200.
 struct VariantRule {
   int d, causal, sk_lo, sk_hi, variant;
 };
@@ -123,16 +116,25 @@ int select_variant(int D, int causal, int Sk) {
   return 0;
 }
 
-template <int kD>
-bool set_smem_attributes() {
-  const int bytes = static_cast<int>(fwd_smem_bytes(kD));
-  for (int v = 0; v < kNumVariants; ++v)
-    if (cudaFuncSetAttribute(fused_kernel<kD>(v), cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             bytes) != cudaSuccess)
+// every kernel checks 1 KiB alignment of its dynamic shared memory base
+bool set_smem_attributes(int D) {
+  for (int v = 0; v < kNumVariants; ++v) {
+    const KernelChoice& k = kernel_choice(D, v);
+    if (cudaFuncSetAttribute(k.fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(k.smem)) != cudaSuccess)
       return false;
-  return cudaFuncSetAttribute(attn_fwd_kernel<1, kD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              bytes) == cudaSuccess;
+  }
+  return true;
 }
+
+// ---------------------------------------------------------------------------
+// per-device setup
+// ---------------------------------------------------------------------------
+// 0 = not done, 1 = ok, 2 = unsupported device.
+std::atomic<int> g_dev_state[kMaxDevices];
+int g_dev_sms[kMaxDevices];
+int g_dev_l2[kMaxDevices];
+std::mutex g_dev_mutex;
 
 attn_status device_setup(int* dev_out) {
   int dev = 0;
@@ -154,32 +156,53 @@ attn_status device_setup(int* dev_out) {
       return ATTN_ERR_UNSUPPORTED;
     }
     if (cudaDeviceGetAttribute(&g_dev_sms[dev], cudaDevAttrMultiProcessorCount, dev) !=
-        cudaSuccess)
+            cudaSuccess ||
+        cudaDeviceGetAttribute(&g_dev_l2[dev], cudaDevAttrL2CacheSize, dev) != cudaSuccess)
       return ATTN_ERR_CUDA;
-    if (!set_smem_attributes<128>() || !set_smem_attributes<64>() ||
-        cudaFuncSetAttribute(pair::attn_fwd_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(pair_smem_bytes())) != cudaSuccess)
+    if (!set_smem_attributes(128) || !set_smem_attributes(64) || !set_smem_attributes(256))
       return ATTN_ERR_CUDA;
-    if (kPairFusedPass) {
-      // a persistent grid of as many CTA pairs as can be resident together
-      cudaLaunchConfig_t cfg = {};
-      cfg.gridDim = dim3(2 * (g_dev_sms[dev] / 2));
-      cfg.blockDim = dim3(pair::kThreads);
-      cfg.dynamicSmemBytes = pair_smem_bytes();
-      int pairs = 0;
-      if (cudaOccupancyMaxActiveClusters(&pairs, pair::attn_fwd_pair_kernel, &cfg) !=
-              cudaSuccess ||
-          pairs < 1)
-        return ATTN_ERR_CUDA;
-      g_dev_pairs[dev] = pairs;
-    }
     g_dev_state[dev].store(1, std::memory_order_release);
   }
   return g_dev_state[dev].load() == 1 ? ATTN_OK : ATTN_ERR_UNSUPPORTED;
 }
 
-// 2-D view [rows, D] fp16 of a dense [.., S, D] tensor; 64 x box_rows boxes
-// (one 128-byte swizzle panel).
+// ---------------------------------------------------------------------------
+// status blocks: kStatusWords words of device memory per (device, stream),
+// zeroed on that stream when created.  The legacy default stream (0) is one
+// stream shared by every host thread; cudaStreamPerThread names a different
+// stream in each host thread, so it gets one block per (device, thread).
+// ---------------------------------------------------------------------------
+using StatusKey = std::tuple<int, cudaStream_t, std::thread::id>;
+std::map<StatusKey, unsigned int*> g_status_blocks;
+std::mutex g_status_mutex;
+
+StatusKey status_key(int dev, cudaStream_t stream) {
+  const bool per_thread = stream == cudaStreamPerThread;
+  return StatusKey(dev, stream, per_thread ? std::this_thread::get_id() : std::thread::id());
+}
+
+unsigned int* status_block(int dev, cudaStream_t stream, bool create) {
+  std::lock_guard<std::mutex> lock(g_status_mutex);
+  const StatusKey key = status_key(dev, stream);
+  auto it = g_status_blocks.find(key);
+  if (it != g_status_blocks.end()) return it->second;
+  if (!create) return nullptr;
+  void* ptr = nullptr;
+  const size_t bytes = kStatusWords * sizeof(unsigned int);
+  if (cudaMalloc(&ptr, bytes) != cudaSuccess) return nullptr;
+  if (cudaMemsetAsync(ptr, 0, bytes, stream) != cudaSuccess) {
+    cudaFree(ptr);
+    return nullptr;
+  }
+  g_status_blocks[key] = static_cast<unsigned int*>(ptr);
+  return static_cast<unsigned int*>(ptr);
+}
+
+// ---------------------------------------------------------------------------
+// launch
+// ---------------------------------------------------------------------------
+// 2-D view [rows, D] fp16 of a dense [.., S, D] tensor; boxes of 64 columns
+// (one 128-byte swizzle panel) x box_rows rows.
 bool encode_rows_map(CUtensorMap* map, const void* base, uint64_t rows, int D,
                      uint32_t box_rows = kBlockM) {
   auto fn = encode_fn();
@@ -195,6 +218,102 @@ bool encode_rows_map(CUtensorMap* map, const void* base, uint64_t rows, int D,
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+attn_status validate_sizes(int B, int Hq, int Hkv, int S, int D, int Sk = -1, int causal = 0) {
+  if (Sk < 0) Sk = S;
+  if (B < 1 || Hq < 1 || Hkv < 1 || S < 1 || Sk < 1 || D < 1) return ATTN_ERR_SHAPE;
+  if (Hq % Hkv != 0) return ATTN_ERR_SHAPE;
+  // a causal query with no visible key (Sq > Sk) has no softmax
+  if (causal && S > Sk) return ATTN_ERR_SHAPE;
+  if (static_cast<int64_t>(B) * Hkv * Sk >= (int64_t(1) << 31)) return ATTN_ERR_SHAPE;
+  if (D != 64 && D != 128 && D != 256) return ATTN_ERR_UNSUPPORTED;
+  // row indices are 32-bit signed in the kernel and in TMA coordinates
+  const int64_t q_rows = static_cast<int64_t>(B) * Hq * S;
+  if (q_rows >= (int64_t(1) << 31)) return ATTN_ERR_SHAPE;
+  return ATTN_OK;
+}
+
+attn_status validate_pointers(const void* q, const void* k, const void* v, const void* o,
+                              const float* lse) {
+  if (!q || !k || !v || !o || !lse) return ATTN_ERR_NULL;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u) != 0)
+    return ATTN_ERR_ALIGN;
+  return ATTN_OK;
+}
+
+size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+// Kernel parameters of one launch over B batch elements (Sq query rows over
+// Sk keys) on a device with `sms` SMs and `l2` bytes of L2.
+FwdParams make_params(void* o, float* lse, unsigned int* status, int B, int Hq, int Hkv, int Sq,
+                      int Sk, int D, int causal, int sms, int l2, bool one_tile) {
+  FwdParams p;
+  p.o = static_cast<__half*>(o);
+  p.lse = lse;
+  p.status = status;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.S = Sq;
+  p.Sk = Sk;
+  p.causal = causal ? 1 : 0;
+  p.off = causal ? Sk - Sq : 0;
+  p.n_qb = (Sq + kBlockM - 1) / kBlockM;
+  p.n_kb = (Sk + kBlockN - 1) / kBlockN;
+  p.group = Hq / Hkv;
+  // 256-row items (two tiles sharing each K/V tile) unless the kernel takes
+  // one tile per item, or two-tile items would leave SMs idle
+  const long long heads = static_cast<long long>(B) * Hq;
+  p.item_tiles = (one_tile || heads * ((p.n_qb + 1) / 2) < sms) ? 1 : 2;
+  p.n_qi = (p.n_qb + p.item_tiles - 1) / p.item_tiles;
+  p.n_items = static_cast<int>(heads * p.n_qi);
+  // Longest first (snake) balances a causal launch; it walks all kv heads at
+  // once, so it is used only when all of K and V stay resident in L2.
+  const double kv_bytes = 2.0 * B * Hkv * static_cast<double>(Sk) * D * 2;
+  p.order = (causal && kv_bytes <= 0.5 * l2) ? 1 : 0;
+  p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
+  p.timeout_ns = g_timeout_ns.load();
+  return p;
+}
+
+// One call: the batch is split into launches of at most kMaxItemsPerCta
+// items per CTA (the exact pass's bit set), each with its own tensor maps.
+attn_status launch_call(const void* q, const void* k, const void* v, void* o, float* lse,
+                        unsigned int* status, int B, int Hq, int Hkv, int Sq, int Sk, int D,
+                        int causal, int variant, int dev, cudaStream_t cs) {
+  const int sms = g_dev_sms[dev];
+  const KernelChoice& kc = kernel_choice(D, variant);
+  const FwdParams whole = make_params(o, lse, status, B, Hq, Hkv, Sq, Sk, D, causal, sms,
+                                      g_dev_l2[dev], kc.one_tile != 0);
+  const long long per_b = static_cast<long long>(whole.n_items) / B;
+  const long long max_items = static_cast<long long>(sms) * kMaxItemsPerCta;
+  const int chunk_b = static_cast<int>(per_b >= max_items ? 1 : max_items / per_b);
+  if (per_b > max_items) return ATTN_ERR_SHAPE;  // one batch element would not fit
+  const size_t q_b = static_cast<size_t>(Hq) * Sq * D;   // elements per batch element
+  const size_t kv_b = static_cast<size_t>(Hkv) * Sk * D;
+  const size_t l_b = static_cast<size_t>(Hq) * Sq;
+  for (int b0 = 0; b0 < B; b0 += chunk_b) {
+    const int nb = B - b0 < chunk_b ? B - b0 : chunk_b;
+    const __half* qc = static_cast<const __half*>(q) + q_b * b0;
+    const __half* kch = static_cast<const __half*>(k) + kv_b * b0;
+    const __half* vc = static_cast<const __half*>(v) + kv_b * b0;
+    __half* oc = static_cast<__half*>(o) + q_b * b0;
+    float* lc = lse + l_b * b0;
+    CUtensorMap tq, tk, tv;
+    const uint32_t kv_box = static_cast<uint32_t>(kc.kv_box);
+    if (!encode_rows_map(&tq, qc, static_cast<uint64_t>(nb) * Hq * Sq, D) ||
+        !encode_rows_map(&tk, kch, static_cast<uint64_t>(nb) * Hkv * Sk, D, kv_box) ||
+        !encode_rows_map(&tv, vc, static_cast<uint64_t>(nb) * Hkv * Sk, D, kv_box))
+      return ATTN_ERR_CUDA;
+    const FwdParams p = make_params(oc, lc, status, nb, Hq, Hkv, Sq, Sk, D, causal, sms,
+                                    g_dev_l2[dev], kc.one_tile != 0);
+    const int grid = p.n_items < sms ? p.n_items : sms;
+    kc.fn<<<grid, kThreads, kc.smem, cs>>>(tq, tk, tv, p);
+    if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  }
+  return ATTN_OK;
+}
 
 // Streams of attn_fwd_host's copy / compute pipeline, created once per device
 // (non-blocking, so they do not serialize with the legacy default stream).
@@ -220,97 +339,63 @@ HostPipe* host_pipe(int dev) {
   return g_host_pipe[dev];
 }
 
-attn_status validate_sizes(int B, int Hq, int Hkv, int S, int D, int Sk = -1, int causal = 0) {
-  if (Sk < 0) Sk = S;
-  if (B < 1 || Hq < 1 || Hkv < 1 || S < 1 || Sk < 1 || D < 1) return ATTN_ERR_SHAPE;
-  if (Hq % Hkv != 0) return ATTN_ERR_SHAPE;
-  // a causal query with no visible key (Sq > Sk) has no softmax
-  if (causal && S > Sk) return ATTN_ERR_SHAPE;
-  if (static_cast<int64_t>(B) * Hkv * Sk >= (int64_t(1) << 31)) return ATTN_ERR_SHAPE;
-  if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
-  // row indices are 32-bit signed in the kernel and in TMA coordinates
-  const int64_t q_rows = static_cast<int64_t>(B) * Hq * S;
-  if (q_rows >= (int64_t(1) << 31)) return ATTN_ERR_SHAPE;
-  if (Hq > 65535 || B > 65535) return ATTN_ERR_SHAPE;  // grid y / z limits
-  return ATTN_OK;
-}
+// ---------------------------------------------------------------------------
+// attn_fwd_noalloc's fixed scratch: the status block lives in this file-scope
+// array instead of memory from cudaMalloc.  Every device that loads the
+// library holds one copy until the process exits.
+// ---------------------------------------------------------------------------
+static __device__ __align__(256) unsigned int g_noalloc_status[kStatusWords];
 
-size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+// Device address of g_noalloc_status, looked up once per device with that
+// device current (host code cannot use the symbol itself as an address).
+unsigned int* g_noalloc_ptr[kMaxDevices];
+std::mutex g_noalloc_mutex;
 
-// Kernel parameters of one call (Sq query rows over Sk keys).
-FwdParams make_params(void* o, float* lse, int B, int Hq, int Hkv, int Sq, int Sk, int D,
-                      int causal) {
-  FwdParams p;
-  p.o = static_cast<__half*>(o);
-  p.lse = lse;
-  p.B = B;
-  p.Hq = Hq;
-  p.Hkv = Hkv;
-  p.S = Sq;
-  p.Sk = Sk;
-  p.causal = causal ? 1 : 0;
-  p.off = causal ? Sk - Sq : 0;
-  p.n_qb = (Sq + kBlockM - 1) / kBlockM;
-  p.n_kb = (Sk + kBlockN - 1) / kBlockN;
-  p.s_tail = Sq - (p.n_qb - 1) * kBlockM;
-  p.n_qb2 = (p.n_qb + 1) / 2;
-  p.group = Hq / Hkv;
-  p.n_items = B * Hq * p.n_qb2;
-  p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
-  p.timeout_ns = g_timeout_ns.load();
-  return p;
-}
-
-// Tensor maps of one call: Q and V in 128-row boxes, K in 64-row boxes (the
-// pair pass loads half a key block per CTA) and 128-row boxes (redo pass).
-struct CallMaps {
-  CUtensorMap q, k, k_half, v;
-};
-
-bool encode_call_maps(CallMaps* m, const void* q, const void* k, const void* v, int B, int Hq,
-                      int Hkv, int Sq, int Sk, int D) {
-  const uint64_t q_rows = static_cast<uint64_t>(B) * Hq * Sq;
-  const uint64_t kv_rows = static_cast<uint64_t>(B) * Hkv * Sk;
-  return encode_rows_map(&m->q, q, q_rows, D) && encode_rows_map(&m->k, k, kv_rows, D) &&
-         encode_rows_map(&m->k_half, k, kv_rows, D, kBlockM / 2) &&
-         encode_rows_map(&m->v, v, kv_rows, D);
-}
-
-// The fused pass over every item (in the given variant), then the hi+lo pass
-// over the items it listed.
-template <int kD>
-attn_status launch_passes_d(const CallMaps& m, const FwdParams& p, int variant, int dev,
-                            cudaStream_t cs) {
-  const int sms = g_dev_sms[dev];
-  // the pair kernel takes D = 128, Sq == Sk and whole 128-row blocks only
-  if (kPairFusedPass && kD == 128 && p.S == p.Sk && p.s_tail == kBlockM) {
-    const int pairs = p.n_items < g_dev_pairs[dev] ? p.n_items : g_dev_pairs[dev];
-    pair::attn_fwd_pair_kernel<<<2 * pairs, pair::kThreads, pair_smem_bytes(), cs>>>(
-        m.q, m.k_half, m.v, p);
-  } else {
-    fused_kernel<kD>(variant)<<<p.n_items < sms ? p.n_items : sms, kThreads, fwd_smem_bytes(kD),
-                                cs>>>(m.q, m.k, m.v, p);
+unsigned int* noalloc_scratch(int dev) {
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (!g_noalloc_ptr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_status) != cudaSuccess || !ptr) return nullptr;
+    g_noalloc_ptr[dev] = static_cast<unsigned int*>(ptr);
   }
-  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
-  attn_fwd_kernel<1, kD><<<sms, kThreads, fwd_smem_bytes(kD), cs>>>(m.q, m.k, m.v, p);
-  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
-  return ATTN_OK;
+  return g_noalloc_ptr[dev];
 }
 
-attn_status launch_passes(const CallMaps& m, const FwdParams& p, int D, int variant, int dev,
-                          cudaStream_t cs) {
-  return D == 64 ? launch_passes_d<64>(m, p, variant, dev, cs)
-                 : launch_passes_d<128>(m, p, variant, dev, cs);
+// Reads (blocking) and clears one status block; ORs its flags into `words`.
+bool drain_status_block(unsigned int* block, unsigned int (&words)[kStatusWords]) {
+  unsigned int w[kStatusWords] = {0, 0, 0, 0};
+  if (cudaMemcpy(w, block, sizeof(w), cudaMemcpyDeviceToHost) != cudaSuccess) return false;
+  if (w[0] | w[1] | w[2] | w[3]) {
+    if (cudaMemset(block, 0, sizeof(w)) != cudaSuccess) return false;
+  }
+  words[0] |= w[0];
+  if (words[1] == 0) words[1] = w[1];
+  words[2] += w[2];
+  return true;
+}
+
+attn_status status_of(const unsigned int (&words)[kStatusWords]) {
+  if (words[0] & kStatusSmemAlign) return ATTN_ERR_CUDA;
+  return (words[0] & kStatusTimeout) ? ATTN_ERR_DEVICE_TIMEOUT : ATTN_OK;
 }
 
 }  // namespace
+
+// The status block of `stream` on the current device (created on first
+// use), for the other kernels of this library (the decoder layer's GEMMs).
+unsigned int* stream_status_block(cudaStream_t stream) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  return status_block(dev, stream, true);
+}
+
 }  // namespace attn_b200
 
 using namespace attn_b200;
 
 extern "C" {
 
-int attn_version(void) { return (1 << 16) | 0; }
+int attn_version(void) { return (2 << 16) | 0; }
 
 const char* attn_status_string(attn_status s) {
   switch (s) {
@@ -319,13 +404,11 @@ const char* attn_status_string(attn_status s) {
     case ATTN_ERR_SHAPE: return "ATTN_ERR_SHAPE: invalid or too large sizes";
     case ATTN_ERR_ALIGN: return "ATTN_ERR_ALIGN: a device pointer is not 16-byte aligned";
     case ATTN_ERR_UNSUPPORTED:
-      return "ATTN_ERR_UNSUPPORTED: needs D == 64 or 128 and an sm_100 device";
+      return "ATTN_ERR_UNSUPPORTED: needs D == 64, 128 or 256 and an sm_100 device";
     case ATTN_ERR_CUDA: return "ATTN_ERR_CUDA: a CUDA call failed";
     case ATTN_ERR_DEVICE_TIMEOUT: return "ATTN_ERR_DEVICE_TIMEOUT: a kernel wait ran out";
     case ATTN_ERR_WORKSPACE: return "ATTN_ERR_WORKSPACE: device workspace too small";
-    case ATTN_ERR_TOO_LARGE:
-      return "ATTN_ERR_TOO_LARGE: B*Hq*ceil(S/256) exceeds attn_fwd_noalloc's fixed scratch "
-             "(131072 work items)";
+    case ATTN_ERR_TOO_LARGE: return "ATTN_ERR_TOO_LARGE: more work than a fixed buffer holds";
   }
   return "ATTN_ERR_UNKNOWN";
 }
@@ -338,11 +421,15 @@ uint64_t attn_set_wait_timeout_ns(uint64_t ns) {
 int attn_variant_count(void) { return kNumVariants; }
 
 const char* attn_variant_name(int variant) {
-  static char names[kNumVariants][48];
+  static char names[kNumVariants][64];
   static std::once_flag once;
   std::call_once(once, [] {
+    static const char* kStructureNames[kStructures] = {
+        "pingpong,mma_issuers=1", "pingpong,mma_issuers=2", "dbuf,softmax_split=1",
+        "dbuf,softmax_split=2"};
     for (int v = 0; v < kNumVariants; ++v)
-      std::snprintf(names[v], sizeof(names[v]), "fma_exp2_pairs=%d/8", kEmuChoices[v]);
+      std::snprintf(names[v], sizeof(names[v]), "%s,fma_exp2_pairs=%d/8",
+                    kStructureNames[variant_structure(v)], variant_emu(v));
   });
   return (variant >= 0 && variant < kNumVariants) ? names[variant] : nullptr;
 }
@@ -355,26 +442,18 @@ int attn_variant_select(int B, int Hq, int Hkv, int Sq, int Sk, int D, int causa
 attn_status attn_fwd_variant(const void* q, const void* k, const void* v, void* o, float* lse,
                              int B, int Hq, int Hkv, int Sq, int Sk, int D, int causal,
                              int variant, void* stream) {
-  if (!q || !k || !v || !o || !lse) return ATTN_ERR_NULL;
-  attn_status st = validate_sizes(B, Hq, Hkv, Sq, D, Sk, causal);
+  attn_status st = validate_pointers(q, k, v, o, lse);
+  if (st != ATTN_OK) return st;
+  st = validate_sizes(B, Hq, Hkv, Sq, D, Sk, causal);
   if (st != ATTN_OK) return st;
   if (variant < 0 || variant >= kNumVariants) return ATTN_ERR_UNSUPPORTED;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
-      (reinterpret_cast<uintptr_t>(lse) & 3u) != 0)
-    return ATTN_ERR_ALIGN;
   int dev = 0;
   st = device_setup(&dev);
   if (st != ATTN_OK) return st;
-
-  CallMaps maps;
-  if (!encode_call_maps(&maps, q, k, v, B, Hq, Hkv, Sq, Sk, D)) return ATTN_ERR_CUDA;
-  FwdParams p = make_params(o, lse, B, Hq, Hkv, Sq, Sk, D, causal);
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
-  p.redo = redo_list(dev, cs);
-  if (!p.redo) return ATTN_ERR_CUDA;
-  p.redo_capacity = kRedoCapacity;
-
-  return launch_passes(maps, p, D, variant, dev, cs);
+  unsigned int* status = status_block(dev, cs, true);
+  if (!status) return ATTN_ERR_CUDA;
+  return launch_call(q, k, v, o, lse, status, B, Hq, Hkv, Sq, Sk, D, causal, variant, dev, cs);
 }
 
 attn_status attn_fwd_qk(const void* q, const void* k, const void* v, void* o, float* lse, int B,
@@ -396,18 +475,23 @@ size_t attn_fwd_host_workspace_bytes(int B, int Hq, int Hkv, int S, int D) {
   return round256(q) * 2 + round256(kv) * 2 + round256(l);
 }
 
-attn_status attn_device_status(void* stream, uint32_t* site) {
+attn_status attn_device_status_ex(void* stream, uint32_t* site, uint64_t* exact_items) {
   if (site) *site = 0;
-  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return ATTN_ERR_CUDA;
-  unsigned int words[2] = {0, 0};
-  if (cudaMemcpyFromSymbol(words, g_attn_status, sizeof(words)) != cudaSuccess) return ATTN_ERR_CUDA;
-  if (words[0] != 0 || words[1] != 0) {
-    const unsigned int zero[2] = {0, 0};
-    if (cudaMemcpyToSymbol(g_attn_status, zero, sizeof(zero)) != cudaSuccess) return ATTN_ERR_CUDA;
-  }
+  if (exact_items) *exact_items = 0;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(cs) != cudaSuccess) return ATTN_ERR_CUDA;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ATTN_ERR_CUDA;
+  unsigned int words[kStatusWords] = {0, 0, 0, 0};
+  unsigned int* block = status_block(dev, cs, false);
+  if (block && !drain_status_block(block, words)) return ATTN_ERR_CUDA;
   if (site) *site = words[1];
-  if (words[0] & kStatusSmemAlign) return ATTN_ERR_CUDA;
-  return (words[0] & kStatusTimeout) ? ATTN_ERR_DEVICE_TIMEOUT : ATTN_OK;
+  if (exact_items) *exact_items = words[2];
+  return status_of(words);
+}
+
+attn_status attn_device_status(void* stream, uint32_t* site) {
+  return attn_device_status_ex(stream, site, nullptr);
 }
 
 attn_status attn_fwd_host(const void* q_h, const void* k_h, const void* v_h, void* o_h,
@@ -493,7 +577,9 @@ attn_status attn_fwd_host(const void* q_h, const void* k_h, const void* v_h, voi
   if (cudaEventRecord(ev_end, hp->down) != cudaSuccess ||
       cudaStreamWaitEvent(cs, ev_end, 0) != cudaSuccess)
     return fail(ATTN_ERR_CUDA);
-  st = attn_device_status(stream, nullptr);
+  if (cudaStreamSynchronize(cs) != cudaSuccess) return fail(ATTN_ERR_CUDA);
+  // the kernels ran on the pipeline's compute stream: report its status
+  st = attn_device_status(hp->comp, nullptr);
   for (int i = 0; i < n_ev; ++i) cudaEventDestroy(ev[i]);
   return st;
 }
@@ -502,8 +588,8 @@ attn_status attn_fwd_host(const void* q_h, const void* k_h, const void* v_h, voi
 
 namespace attn_b200 {
 // One thread waits, with the kernels' bounded wait, on an mbarrier that no
-// one arrives on.
-__global__ void selftest_wait_kernel(uint64_t timeout_ns) {
+// one arrives on, and records the timeout in `status`.
+__global__ void selftest_wait_kernel(uint64_t timeout_ns, unsigned int* status) {
   __shared__ uint64_t bar;
   __shared__ int abort_flag;
   if (threadIdx.x == 0) {
@@ -512,11 +598,9 @@ __global__ void selftest_wait_kernel(uint64_t timeout_ns) {
     fence_mbar_init();
   }
   __syncthreads();
-  if (threadIdx.x == 0) mbar_wait(smem_addr(&bar), 0, &abort_flag, timeout_ns, 0x501);
+  if (threadIdx.x == 0) mbar_wait(smem_addr(&bar), 0, &abort_flag, timeout_ns, status, 0x501);
 }
-}  // namespace attn_b200
 
-namespace attn_b200 {
 // The fast pass's FMA-pipe exponential, evaluated elementwise (pairs).
 __global__ void selftest_exp2_kernel(const float* x, float* y, int n) {
   const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
@@ -546,71 +630,47 @@ extern "C" attn_status attn_selftest_wait_timeout(uint64_t timeout_ns, void* str
   int dev = 0;
   attn_status st = device_setup(&dev);
   if (st != ATTN_OK) return st;
-  selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(timeout_ns);
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  unsigned int* status = status_block(dev, cs, true);
+  if (!status) return ATTN_ERR_CUDA;
+  selftest_wait_kernel<<<1, 32, 0, cs>>>(timeout_ns, status);
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
   return attn_device_status(stream, nullptr);
 }
 
 // ---------------------------------------------------------------------------
-// attn_fwd_noalloc: the same two launches as attn_fwd, with the redo list in
-// a fixed array of this file instead of memory from cudaMalloc.
+// attn_fwd_noalloc: the same launches as attn_fwd, with the call's status
+// block in this file's fixed array instead of memory from cudaMalloc.
 // ---------------------------------------------------------------------------
-namespace attn_b200 {
-namespace {
-
-constexpr unsigned int kNoAllocMaxItems = 1u << 17;  // 131072 items: 512 KiB of ids
-
-// Header {count, done, -, -} then up to kNoAllocMaxItems item ids.  Every
-// device that loads the library holds one copy until the process exits.
-static __device__ __align__(256) unsigned int g_noalloc_redo[kRedoHeaderWords + kNoAllocMaxItems];
-
-// Device address of g_noalloc_redo, looked up once per device with that
-// device current (host code cannot use the symbol itself as an address).
-unsigned int* g_noalloc_ptr[kMaxDevices];
-std::mutex g_noalloc_mutex;
-
-unsigned int* noalloc_scratch(int dev) {
-  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-  if (!g_noalloc_ptr[dev]) {
-    void* ptr = nullptr;
-    if (cudaGetSymbolAddress(&ptr, g_noalloc_redo) != cudaSuccess || !ptr) return nullptr;
-    g_noalloc_ptr[dev] = static_cast<unsigned int*>(ptr);
-  }
-  return g_noalloc_ptr[dev];
-}
-
-}  // namespace
-}  // namespace attn_b200
-
 extern "C" attn_status attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o,
                                         float* lse, int B, int Hq, int Hkv, int S, int D,
                                         int causal, void* stream) {
-  if (!q || !k || !v || !o || !lse) return ATTN_ERR_NULL;
-  attn_status st = validate_sizes(B, Hq, Hkv, S, D);
+  attn_status st = validate_pointers(q, k, v, o, lse);
   if (st != ATTN_OK) return st;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
-      (reinterpret_cast<uintptr_t>(lse) & 3u) != 0)
-    return ATTN_ERR_ALIGN;
-  const int n_qb = (S + kBlockM - 1) / kBlockM;
-  const int n_qb2 = (n_qb + 1) / 2;
-  const long long n_items = static_cast<long long>(B) * Hq * n_qb2;
-  if (n_items > kNoAllocMaxItems) return ATTN_ERR_TOO_LARGE;
+  st = validate_sizes(B, Hq, Hkv, S, D);
+  if (st != ATTN_OK) return st;
   int dev = 0;
   st = device_setup(&dev);
   if (st != ATTN_OK) return st;
   unsigned int* scratch = noalloc_scratch(dev);
   if (!scratch) return ATTN_ERR_CUDA;
-
-  CallMaps maps;
-  if (!encode_call_maps(&maps, q, k, v, B, Hq, Hkv, S, S, D)) return ATTN_ERR_CUDA;
-
-  FwdParams p = make_params(o, lse, B, Hq, Hkv, S, S, D, causal);
-  p.redo = scratch;
-  p.redo_capacity = kNoAllocMaxItems;  // >= n_items: the list cannot overflow
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  return launch_call(q, k, v, o, lse, scratch, B, Hq, Hkv, S, S, D, causal,
+                     select_variant(D, causal, S), dev, cs);
+}
 
-  // the shared array keeps the previous call's header: start from an empty list
-  if (cudaMemsetAsync(scratch, 0, kRedoHeaderWords * sizeof(unsigned int), cs) != cudaSuccess)
+extern "C" attn_status attn_noalloc_status(void* stream, uint32_t* site, uint64_t* exact_items) {
+  if (site) *site = 0;
+  if (exact_items) *exact_items = 0;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return ATTN_ERR_CUDA;
-  return launch_passes(maps, p, D, select_variant(D, causal, S), dev, cs);
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ATTN_ERR_CUDA;
+  unsigned int* scratch = noalloc_scratch(dev);
+  if (!scratch) return ATTN_ERR_CUDA;
+  unsigned int words[kStatusWords] = {0, 0, 0, 0};
+  if (!drain_status_block(scratch, words)) return ATTN_ERR_CUDA;
+  if (site) *site = words[1];
+  if (exact_items) *exact_items = words[2];
+  return status_of(words);
 }

@@ -1,7 +1,7 @@
 // ptx_sm100.cuh -- inline-PTX building blocks for sm_100a: mbarriers with
 // time-bounded waits, TMA tile loads, tcgen05 (tensor-core MMA, TMEM
-// allocation, TMEM loads/stores, commits) and the shared-memory / instruction
-// descriptors the MMAs read.
+// allocation, TMEM loads/stores, commits), the shared-memory / instruction
+// descriptors the MMAs read, and the few arithmetic forms the softmax needs.
 //
 // These are the B200 counterparts of the pages' specialised execution units
 // (papers.lqhl.me "PipeThreader-OSDI25", section 核心方法, "sTask / sEU": a
@@ -15,9 +15,9 @@
 
 namespace attn_b200 {
 
-// --------------------------------------------------------------------------
-// generic helpers
-// --------------------------------------------------------------------------
+// ===========================================================================
+// generic
+// ===========================================================================
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
@@ -28,9 +28,46 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
   return t;
 }
 
-// --------------------------------------------------------------------------
+// One lane of a converged warp (the same lane every time): 1 there, 0 in the
+// other lanes.
+__device__ __forceinline__ uint32_t elect_one() {
+  uint32_t e;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "elect.sync _|p, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(e));
+  return e;
+}
+
+// Register reallocation between warpgroups (every warp of a warpgroup
+// executes the same one).
+template <int kRegs>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegs));
+}
+template <int kRegs>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegs));
+}
+
+// ===========================================================================
+// per-call status block (device memory the host gives each launch)
+//   [0] error flags, [1] first wait site that ran out, [2] items recomputed
+//   by the exact pass, [3] reserved
+// ===========================================================================
+constexpr int kStatusWords = 4;
+constexpr unsigned int kStatusTimeout = 1u;
+constexpr unsigned int kStatusSmemAlign = 2u;  // dynamic shared memory base not 1 KiB aligned
+
+__device__ __forceinline__ void record_timeout(unsigned int* status, uint32_t site) {
+  atomicOr(&status[0], kStatusTimeout);
+  atomicCAS(&status[1], 0u, site);
+}
+
+// ===========================================================================
 // mbarriers
-// --------------------------------------------------------------------------
+// ===========================================================================
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
 }
@@ -49,6 +86,8 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
                : "memory");
 }
 
+// Potentially blocking test: the thread may be suspended for a while if the
+// phase is not complete yet.
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
@@ -61,56 +100,63 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Device-wide status words of this library: [0] error flags, [1] first wait
-// site that ran out.  The library is a single translation unit, which owns
-// this definition; the host reads it with cudaMemcpyFromSymbol.
-__device__ unsigned int g_attn_status[2];
-constexpr unsigned int kStatusTimeout = 1u;
-constexpr unsigned int kStatusSmemAlign = 2u;  // dynamic shared memory base not 1 KiB aligned
+// Non-blocking test.
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
 
 // Waits until phase `parity` of the barrier has completed.  Bounded: after
 // `timeout_ns` of wall time, or as soon as another role of the CTA has given
-// up (*abort != 0), it records the failure and returns false so the caller
-// can wind down instead of hanging.  The fast path is a plain try_wait.
+// up (*abort != 0), it records the failure in `status` and returns false so
+// the caller can wind down instead of hanging.  kSpin selects non-blocking
+// polling (lowest wake-up latency, for the one thread that feeds the tensor
+// core) instead of the suspending test.
+template <bool kSpin = false>
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort,
-                                          uint64_t timeout_ns, uint32_t site) {
-  if (mbar_try_wait(bar, parity)) return true;
+                                          uint64_t timeout_ns, unsigned int* status,
+                                          uint32_t site) {
+  if (kSpin ? mbar_test_wait(bar, parity) : mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   while (true) {
 #pragma unroll 1
-    for (int i = 0; i < 32; ++i)
-      if (mbar_try_wait(bar, parity)) return true;
+    for (int i = 0; i < 64; ++i)
+      if (kSpin ? mbar_test_wait(bar, parity) : mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
     if (global_timer_ns() - t0 > timeout_ns) {
       *abort = 1;
-      atomicOr(&g_attn_status[0], kStatusTimeout);
-      atomicCAS(&g_attn_status[1], 0u, site);
+      record_timeout(status, site);
       return false;
     }
   }
 }
 
-// --------------------------------------------------------------------------
+// Waits (bounded, ignoring the abort flag) for copies or MMAs in flight to
+// land before a CTA that gave up exits.
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64_t timeout_ns,
+                                           unsigned int* status, uint32_t site = 0x501) {
+  int never = 0;
+  mbar_wait(bar, parity, &never, timeout_ns, status, site);
+}
+
+// ===========================================================================
 // TMA (tiled bulk tensor copies, global -> shared), no multicast
-// --------------------------------------------------------------------------
+// ===========================================================================
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
 // Loads the box at element coordinates (x = column, y = row) into `dst`,
-// completing `bytes` of transaction count on `bar`.
+// completing its bytes on `bar`, with an L2 eviction-priority policy.
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
-                                            int32_t x, int32_t y) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y)
-      : "memory");
-}
-
-// Same, with an L2 eviction-priority policy (createpolicy result).
-__device__ __forceinline__ void tma_load_2d_hint(uint32_t dst, const CUtensorMap* map, uint32_t bar,
-                                                 int32_t x, int32_t y, uint64_t policy) {
+                                            int32_t x, int32_t y, uint64_t policy) {
   asm volatile(
       "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
       " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(dst),
@@ -130,9 +176,9 @@ __device__ __forceinline__ uint64_t l2_policy_evict_first() {
   return p;
 }
 
-// --------------------------------------------------------------------------
-// tcgen05: TMEM allocation, fences, MMA, commit, TMEM <-> registers
-// --------------------------------------------------------------------------
+// ===========================================================================
+// tcgen05: TMEM allocation, fences, MMA, commit
+// ===========================================================================
 // One full warp executes alloc/dealloc.  The allocated base (lane 0, first
 // column) is written to shared memory at `dst`.
 __device__ __forceinline__ void tmem_alloc(uint32_t dst, uint32_t ncols) {
@@ -155,38 +201,62 @@ __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
-// D[tmem] (+)= A[smem desc] * B[smem desc]^T, kind::f16, one CTA.
-__device__ __forceinline__ void mma_f16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                           uint32_t idesc, uint32_t accumulate) {
+// The MMA and commit forms below are executed by a whole converged warp; one
+// elected lane issues the operation.  Keeping the issuing code warp-uniform
+// lets the descriptors live in uniform registers.
+//
+// D[tmem] (+)= A[smem desc + kOffA] * B[smem desc + kOffB]^T, kind::f16.
+// Descriptor offsets are in 16-byte units (the start-address field of the
+// descriptor, which never carries out for addresses below 256 KiB).
+template <uint32_t kOffA, uint32_t kOffB>
+__device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                       uint32_t idesc, uint32_t accumulate) {
   asm volatile(
-      "{\n\t.reg .pred p;\n\t"
+      "{\n\t.reg .pred p, e;\n\t.reg .b64 da, db;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "add.s64 da, %1, %5;\n\t"
+      "add.s64 db, %2, %6;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "n"(kOffA), "n"(kOffB)
       : "memory");
 }
 
-// D[tmem] (+)= A[tmem] * B[smem desc], kind::f16, one CTA.
-__device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                           uint32_t idesc, uint32_t accumulate) {
+// D[tmem] (+)= A[tmem + kOffA columns] * B[smem desc + kOffB], kind::f16.
+template <uint32_t kOffA, uint32_t kOffB>
+__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                       uint32_t idesc, uint32_t accumulate) {
   asm volatile(
-      "{\n\t.reg .pred p;\n\t"
+      "{\n\t.reg .pred p, e;\n\t.reg .b64 db;\n\t.reg .b32 ta;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "add.u32 ta, %1, %5;\n\t"
+      "add.s64 db, %2, %6;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], db, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate), "n"(kOffA), "n"(kOffB)
       : "memory");
 }
 
-// Arrives once on `bar` when every tcgen05 operation this thread issued
+// Arrives once on `bar` when every tcgen05 operation the elected lane issued
 // before it has completed.
 __device__ __forceinline__ void tc_commit(uint32_t bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                   bar)
-               : "memory");
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(
+          bar)
+      : "memory");
 }
 
+// ===========================================================================
+// tcgen05: TMEM <-> registers (32x32b shapes: thread t of the warp holds
+// lane (base lane + t), consecutive 32-bit columns)
+// ===========================================================================
 __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
 // tcgen05.ld writes its destination registers asynchronously: they hold the
@@ -206,13 +276,18 @@ __device__ __forceinline__ void reg_dep32(uint32_t* r) {
   reg_dep16(r);
   reg_dep16(r + 16);
 }
-__device__ __forceinline__ void tmem_wait_st() {
-  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
 }
 
-// 32 lanes x 32 consecutive 32-bit columns: thread t of the warp receives
-// lane (base lane + t), columns [col, col + 32).
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t* r) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
       "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
@@ -225,7 +300,14 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
       : "r"(taddr));
 }
 
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
       "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
@@ -239,9 +321,9 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
       : "memory");
 }
 
-// --------------------------------------------------------------------------
+// ===========================================================================
 // descriptors
-// --------------------------------------------------------------------------
+// ===========================================================================
 // Shared-memory matrix descriptor (tcgen05 format, version 1) for a 128-byte
 // swizzled layout.  Start address, leading-dimension byte offset (LBO) and
 // stride-dimension byte offset (SBO) are stored in 16-byte units.
@@ -273,9 +355,9 @@ __host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N, bool a_mn, bo
          | (static_cast<uint32_t>(M >> 4) << 24);  // M / 16
 }
 
-// --------------------------------------------------------------------------
+// ===========================================================================
 // arithmetic
-// --------------------------------------------------------------------------
+// ===========================================================================
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -290,9 +372,6 @@ __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
   return r;
 }
 
-}  // namespace attn_b200
-
-namespace attn_b200 {
 // acc + lo(h2) + hi(h2), where lo/hi are the two fp16 halves of h2 widened
 // exactly to fp32 (mixed-precision add, no separate conversion).
 __device__ __forceinline__ float add_half2_f32(uint32_t h2, float acc) {
@@ -304,91 +383,7 @@ __device__ __forceinline__ float add_half2_f32(uint32_t h2, float acc) {
       : "r"(h2));
   return acc;
 }
-}  // namespace attn_b200
 
-namespace attn_b200 {
-// Register reallocation between warpgroups (all warps of a warpgroup execute
-// the same one).
-template <int kRegs>
-__device__ __forceinline__ void regs_inc() {
-  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegs));
-}
-template <int kRegs>
-__device__ __forceinline__ void regs_dec() {
-  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegs));
-}
-
-// Named barrier over `count` threads (id 0 is __syncthreads).
-__device__ __forceinline__ void named_barrier(int id, int count) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
-}
-
-// 32 lanes x 16 consecutive 32-bit columns.
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
-      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
-      "r"(r[15])
-      : "memory");
-}
-}  // namespace attn_b200
-
-namespace attn_b200 {
-// 32 lanes x 8 consecutive 32-bit columns.
-__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
-      : "memory");
-}
-}  // namespace attn_b200
-
-namespace attn_b200 {
-// 32 lanes x 16 consecutive 32-bit columns.
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-        "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr));
-}
-}  // namespace attn_b200
-
-namespace attn_b200 {
-// As mma_f16_ss / mma_f16_ts, with compile-time byte offsets (in 16-byte
-// units) added to the descriptors inside the instruction block, so callers
-// keep only the base descriptors live.
-template <uint32_t kOffA, uint32_t kOffB>
-__device__ __forceinline__ void mma_f16_ss_off(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                               uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t.reg .b64 da, db;\n\t"
-      "add.s64 da, %1, %5;\n\t"
-      "add.s64 db, %2, %6;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "n"(kOffA), "n"(kOffB)
-      : "memory");
-}
-template <uint32_t kOffA, uint32_t kOffB>
-__device__ __forceinline__ void mma_f16_ts_off(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                               uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t.reg .b64 db;\n\t.reg .b32 ta;\n\t"
-      "add.u32 ta, %1, %5;\n\t"
-      "add.s64 db, %2, %6;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], db, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate), "n"(kOffA), "n"(kOffB)
-      : "memory");
-}
-}  // namespace attn_b200
-
-namespace attn_b200 {
 // max(a, b, c) in one instruction.
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;
@@ -421,177 +416,5 @@ __device__ __forceinline__ float2 exp2_poly2(float2 x) {
   return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
                      __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
 }
-}  // namespace attn_b200
 
-namespace attn_b200 {
-// 32 lanes x 64 consecutive 32-bit columns in one instruction.
-__device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x64.b32 "
-      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
-      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, "
-      "%32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, "
-      "%48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63}, [%64];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
-        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
-        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]),
-        "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]),
-        "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]),
-        "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]),
-        "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]),
-        "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]),
-        "=r"(r[62]), "=r"(r[63])
-      : "r"(taddr));
-}
-}  // namespace attn_b200
-
-namespace attn_b200 {
-// --------------------------------------------------------------------------
-// CTA pairs (a 2-CTA cluster on two SMs): one tcgen05.mma.cta_group::2 spans
-// both SMs, M = 256 (each CTA holds 128 rows of A and of the accumulator in
-// its own TMEM, and half of B's N rows in its own shared memory).  Only the
-// even CTA issues MMAs and commits; the odd one supplies its operands.
-// --------------------------------------------------------------------------
-__device__ __forceinline__ uint32_t cluster_ctarank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-__device__ __forceinline__ uint32_t cluster_nctarank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
-  return r;
-}
-// Address of the same shared-memory offset in CTA `rank` of the cluster.
-__device__ __forceinline__ uint32_t smem_map_rank(uint32_t addr, uint32_t rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
-  return r;
-}
-// Every thread of both CTAs: release own prior writes, wait for the others'.
-__device__ __forceinline__ void cluster_sync() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" :::
-                   "memory");
-}
-__device__ __forceinline__ void st_cluster_u32(uint32_t caddr, uint32_t v) {
-  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(caddr), "r"(v) : "memory");
-}
-
-// TMEM for pair MMAs: the same warp index of both CTAs executes these.
-__device__ __forceinline__ void tmem_alloc_pair(uint32_t dst, uint32_t ncols) {
-  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst),
-               "r"(ncols)
-               : "memory");
-}
-__device__ __forceinline__ void tmem_relinquish_pair() {
-  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
-  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
-               : "memory");
-}
-
-// Pair MMAs with compile-time descriptor offsets (16-byte units for shared
-// memory, columns for TMEM), as mma_f16_ss_off / mma_f16_ts_off.
-template <uint32_t kOffA, uint32_t kOffB>
-__device__ __forceinline__ void mma_pair_ss_off(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                                uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t.reg .b64 da, db;\n\t"
-      "add.s64 da, %1, %5;\n\t"
-      "add.s64 db, %2, %6;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::2.kind::f16 [%0], da, db, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "n"(kOffA), "n"(kOffB)
-      : "memory");
-}
-template <uint32_t kOffA, uint32_t kOffB>
-__device__ __forceinline__ void mma_pair_ts_off(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                                uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t.reg .b64 db;\n\t.reg .b32 ta;\n\t"
-      "add.u32 ta, %1, %5;\n\t"
-      "add.s64 db, %2, %6;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::2.kind::f16 [%0], [ta], db, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate), "n"(kOffA), "n"(kOffB)
-      : "memory");
-}
-// Arrives once on the barrier at offset `bar` of every CTA in `cta_mask`
-// when all pair MMAs this thread issued before it have completed.
-__device__ __forceinline__ void tc_commit_pair(uint32_t bar, uint16_t cta_mask) {
-  asm volatile(
-      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 "
-      "[%0], %1;" ::"r"(bar),
-      "h"(cta_mask)
-      : "memory");
-}
-// Tile load into this CTA's shared memory whose completion (bytes) is
-// counted on `bar`, which may be the even CTA's barrier (no multicast).
-__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, uint32_t bar,
-                                                 int32_t x, int32_t y, uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
-      ".L2::cache_hint [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y), "l"(policy)
-      : "memory");
-}
-// Atomics on a shared-memory word of any CTA of the cluster.
-__device__ __forceinline__ uint32_t atom_add_cluster(uint32_t caddr, uint32_t v) {
-  uint32_t old;
-  asm volatile("atom.acq_rel.cluster.shared::cluster.add.u32 %0, [%1], %2;"
-               : "=r"(old)
-               : "r"(caddr), "r"(v)
-               : "memory");
-  return old;
-}
-__device__ __forceinline__ uint32_t atom_or_cluster(uint32_t caddr, uint32_t v) {
-  uint32_t old;
-  asm volatile("atom.acq_rel.cluster.shared::cluster.or.b32 %0, [%1], %2;"
-               : "=r"(old)
-               : "r"(caddr), "r"(v)
-               : "memory");
-  return old;
-}
-__device__ __forceinline__ uint32_t atom_exch_cluster(uint32_t caddr, uint32_t v) {
-  uint32_t old;
-  asm volatile("atom.acq_rel.cluster.shared::cluster.exch.b32 %0, [%1], %2;"
-               : "=r"(old)
-               : "r"(caddr), "r"(v)
-               : "memory");
-  return old;
-}
-// Arrive on a barrier of either CTA of the pair.  What the arrive publishes
-// is TMEM contents (ordered by tcgen05.wait + tcgen05.fence before it and
-// tcgen05.fence::after_thread_sync after the wait) or the completion of a
-// read, so CTA-scope release suffices; a cluster-scope release would also
-// drain this thread's outstanding memory traffic to cluster scope, which
-// measured about 1000 cycles per arrive.
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t caddr) {
-  asm volatile("mbarrier.arrive.release.cta.shared::cluster.b64 _, [%0];" ::"r"(caddr)
-               : "memory");
-}
-// As mbar_wait; on running out it also raises the other CTA's abort flag
-// (cluster address `peer_abort`).
-__device__ __forceinline__ bool mbar_wait_pair(uint32_t bar, uint32_t parity, volatile int* abort,
-                                               uint32_t peer_abort, uint64_t timeout_ns,
-                                               uint32_t site) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = global_timer_ns();
-  while (true) {
-#pragma unroll 1
-    for (int i = 0; i < 32; ++i)
-      if (mbar_try_wait(bar, parity)) return true;
-    if (*abort) return false;
-    if (global_timer_ns() - t0 > timeout_ns) {
-      *abort = 1;
-      st_cluster_u32(peer_abort, 1u);
-      atomicOr(&g_attn_status[0], kStatusTimeout);
-      atomicCAS(&g_attn_status[1], 0u, site);
-      return false;
-    }
-  }
-}
 }  // namespace attn_b200

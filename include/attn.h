@@ -25,19 +25,22 @@
  *     LSE [B, Hq, S].  "Device" pointers are CUDA device (or managed)
  *     addresses on the current device; "host" pointers are CPU addresses.
  *   - The caller owns every input and output buffer; the library keeps no
- *     pointer to them after returning.  Besides those, attn_fwd (and
- *     attn_fwd_host, which calls it) needs a small device scratch list: the
- *     first call for each (device, stream) pair allocates it with cudaMalloc
- *     (256 KiB + 16 B) and zeroes it on that stream; it is kept for later
- *     calls on that pair until the process exits.  Nothing else allocates.
+ *     pointer to them after returning.  Besides those, the kernels of a call
+ *     write a 16-byte status block (error flags, the first wait that ran out,
+ *     a count of recomputed work items).  The first call for each (device,
+ *     stream) pair allocates that block with cudaMalloc and zeroes it on the
+ *     stream; it is kept for later calls until the process exits.  The
+ *     legacy default stream (NULL) is one stream for every host thread;
+ *     cudaStreamPerThread is a different stream in each host thread, so it
+ *     gets one block per (device, thread).  Nothing else allocates.
  *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls
  *     are asynchronous with respect to the host unless stated otherwise.
  *   - Arguments are validated before anything is launched; a rejected call
  *     launches nothing and leaves the outputs untouched.
  *   - Every wait inside the kernels is bounded in time.  A wait that runs out
  *     makes the kernel stop early (without faulting) and records
- *     ATTN_ERR_DEVICE_TIMEOUT in a per-device status word, read back with
- *     attn_device_status().
+ *     ATTN_ERR_DEVICE_TIMEOUT in the status block of the stream it ran on,
+ *     read back with attn_device_status().
  */
 #ifndef ATTN_B200_H
 #define ATTN_B200_H
@@ -58,7 +61,8 @@ typedef enum attn_status {
   ATTN_ERR_CUDA = 5,           /* a CUDA runtime / driver call failed */
   ATTN_ERR_DEVICE_TIMEOUT = 6, /* a kernel wait ran out; results are invalid */
   ATTN_ERR_WORKSPACE = 7,      /* the device workspace given is too small */
-  ATTN_ERR_TOO_LARGE = 8       /* more work than attn_fwd_noalloc's fixed scratch holds */
+  ATTN_ERR_TOO_LARGE = 8       /* more work than a fixed buffer holds (kept for ABI
+                                  stability; no entry point of this version returns it) */
 } attn_status;
 
 /*
@@ -72,12 +76,14 @@ typedef enum attn_status {
  *   masked).
  *   causal: nonzero for the causal mask j <= i (square, Sq == Sk == S).
  *   stream: cudaStream_t to launch on.
- * Returns ATTN_OK once the kernels are enqueued; errors as listed above.  The
- * outputs must not overlap the inputs.  Two kernels run on `stream`: the
- * fused pass over every 256-row work item, then a pass that recomputes, with
- * probabilities split into two fp16 parts, only the items the first pass
- * listed (those with a row max|O| >= 3.98, where fp16 output rounding leaves
- * almost no error budget); it exits at once when the list is empty.
+ * Returns ATTN_OK once the kernel is enqueued; errors as listed above.  The
+ * outputs must not overlap the inputs.  One kernel runs on `stream` (a call
+ * with more than 2048 work items per SM is split into launches over batch
+ * ranges).  Each CTA of it computes its work items (256 or 128 query rows of
+ * one head) with fp16 probabilities, then recomputes, with the
+ * probabilities split into two fp16 parts, the items that have a row with
+ * max|O| >= 3.98, where fp16 output rounding leaves almost no error budget;
+ * attn_device_status_ex() reports how many items that were.
  */
 attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
                      int B, int Hq, int Hkv, int S, int D, int causal, void* stream);
@@ -90,8 +96,8 @@ attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float
  *   causal: query i sees keys j <= i + (Sk - Sq) (aligned at the bottom right:
  *   the last query sees every key); requires Sq <= Sk (ATTN_ERR_SHAPE
  *   otherwise, as a query would see no key).  Non-causal: any Sq, Sk >= 1.
- * Everything else (pointers, alignment, D, streams, the two launches, errors)
- * is as for attn_fwd, which is attn_fwd_qk with Sq == Sk == S.
+ * Everything else (pointers, alignment, D, streams, launches, errors) is as
+ * for attn_fwd, which is attn_fwd_qk with Sq == Sk == S.
  */
 attn_status attn_fwd_qk(const void* q, const void* k, const void* v, void* o, float* lse,
                         int B, int Hq, int Hkv, int Sq, int Sk, int D, int causal,
@@ -102,16 +108,20 @@ attn_status attn_fwd_qk(const void* q, const void* k, const void* v, void* o, fl
  * is that the best tiling / pipeline choice of an attention kernel is found by
  * profiling candidates on the target GPU (PipeThreader pages, sections 核心方法
  * and 设计取舍: a joint tile + pipeline search whose greedy choices are checked
- * by profiling); this library keeps that idea as a small build-time table.  The fused pass is compiled in
- * attn_variant_count() variants that differ in how many of every 16
- * exponentials of the softmax are evaluated by an FMA-pipe polynomial instead
- * of the MUFU unit (variant i: name "fma_exp2_pairs=N/8", N pairs of 8; all
- * variants compute the same probabilities to within the polynomial's relative
- * error 8e-5, well inside fp16 rounding of P).  The package's tuner
+ * by profiling); this library keeps that idea as a small build-time table.  The fused kernel
+ * is compiled in attn_variant_count() variants along two axes of its
+ * pipeline: how many warps issue the tensor-core MMAs (one for both 128-row
+ * tiles of a work item, or one per tile) and how many of every 16
+ * exponentials of the softmax an FMA-pipe polynomial evaluates instead of the
+ * MUFU unit (variant v: name "mma_issuers=I,fma_exp2_pairs=N/8" with
+ * I = 1 + v / 5, N = v % 5; the issuers axis changes no result, and the
+ * polynomial's relative error 8e-5 is well inside fp16 rounding of P).  The
+ * package's tuner
  * (python -m dnn_compiler_pipelining_b200.tune) times every variant per
  * shape class on a B200 and writes the table compiled into the library;
  * attn_fwd, attn_fwd_qk, attn_fwd_host and attn_fwd_noalloc run the variant
- * the table picks.  The redo pass is the same for every variant.
+ * the table picks.  The exact pass takes every exponential from the MUFU
+ * unit in every variant.
  *
  * attn_variant_count -- number of compiled fused-pass variants (>= 1).
  * attn_variant_name  -- static, human-readable name of a variant; NULL when
@@ -162,12 +172,21 @@ attn_status attn_fwd_host(const void* q_h, const void* k_h, const void* v_h, voi
 
 /*
  * attn_device_status -- synchronizes `stream`, then reads and clears the
- * current device's status word.  Returns ATTN_ERR_DEVICE_TIMEOUT if any
- * kernel of this library recorded a timed-out wait since the last read,
- * ATTN_ERR_CUDA if synchronizing failed, else ATTN_OK.  `site`, if not NULL,
+ * status block of `stream` on the current device (per calling thread for
+ * cudaStreamPerThread).  Returns ATTN_ERR_DEVICE_TIMEOUT if a kernel of this
+ * library launched on that stream recorded a timed-out wait since the last
+ * read, ATTN_ERR_CUDA if synchronizing or reading failed, else ATTN_OK.
+ * Calls on other streams are not reported here.  `site`, if not NULL,
  * receives the first recorded wait site (0 when none).
  */
 attn_status attn_device_status(void* stream, uint32_t* site);
+
+/*
+ * attn_device_status_ex -- attn_device_status, plus `exact_items` (if not
+ * NULL): the number of work items the kernels on `stream` recomputed with
+ * two-part probabilities since the last read.
+ */
+attn_status attn_device_status_ex(void* stream, uint32_t* site, uint64_t* exact_items);
 
 /*
  * attn_set_wait_timeout_ns -- bound, in nanoseconds, on every wait inside the
@@ -188,29 +207,37 @@ attn_status attn_selftest_wait_timeout(uint64_t timeout_ns, void* stream);
 /*
  * attn_fwd_noalloc -- attn_fwd for callers that must not allocate device
  * memory.  No counterpart in the paper: it exists for library users, not for
- * the method.  attn_fwd keeps a small device scratch list per (device,
- * stream) and creates it with cudaMalloc on first use; some callers cannot
- * allow that: serving engines that reserve all device memory up front for
- * their caches, frameworks whose own caching allocator must see every byte,
- * or latency-bound loops where cudaMalloc's implicit device synchronization
- * or a late out-of-memory failure is unacceptable.  This entry point keeps
- * its scratch in a fixed array inside the library instead (512 KiB + 16 B per
- * device, reserved when the library is loaded and held until the process
- * exits), and calls no cudaMalloc, cudaFree or other allocating routine.
- *   Arguments, layouts, results and errors: as attn_fwd, plus
- *   ATTN_ERR_TOO_LARGE when B * Hq * ceil(S / 256) > 131072 (the array's
- *   capacity in 256-row work items; e.g. B=64, Hq=64, S=8192 fits exactly).
+ * the method.  Besides the caller's buffers, the kernel of a call writes a
+ * 16-byte status block; attn_fwd creates one per (device, stream) with
+ * cudaMalloc on first use, and some callers cannot allow that: serving
+ * engines that reserve all device memory up front for their caches,
+ * frameworks whose own caching allocator must see every byte, or
+ * latency-bound loops where cudaMalloc's implicit device synchronization or a
+ * late out-of-memory failure is unacceptable.  This entry point uses a fixed
+ * array inside the library instead (16 bytes per device, reserved when the
+ * library is loaded and held until the process exits), and calls no
+ * cudaMalloc, cudaFree or other allocating routine.
+ *   Arguments, layouts, results and errors: as attn_fwd; the same kernels
+ *   run, so outputs are bit-identical to attn_fwd's.
  *   Set-up: the first call on each device looks up the array's device address
  *   (cudaGetSymbolAddress) with that device current; make that first call
  *   before capturing work into a stream graph.
- *   Sharing: every call on a device uses the same array.  Each call clears its
- *   header on `stream` before launching, so calls ordered on one stream are
- *   independent; calls that overlap on the GPU (different streams, or
- *   different host threads without ordering) race on it and may produce wrong
- *   outputs.
+ *   Sharing: every call on a device writes the same array, which accumulates
+ *   until attn_noalloc_status() reads and clears it.  Calls that overlap on
+ *   the GPU (different streams, or host threads without ordering) mix their
+ *   reports there, so a timeout cannot be attributed to one of them.
  */
 attn_status attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, float* lse,
                              int B, int Hq, int Hkv, int S, int D, int causal, void* stream);
+
+/*
+ * attn_noalloc_status -- synchronizes `stream`, then reads and clears the
+ * fixed status array of attn_fwd_noalloc on the current device: status as
+ * attn_device_status (ATTN_ERR_DEVICE_TIMEOUT if any such call timed out
+ * since the last read), `site` and `exact_items` (if not NULL) as
+ * attn_device_status_ex.  Allocates nothing.
+ */
+attn_status attn_noalloc_status(void* stream, uint32_t* site, uint64_t* exact_items);
 
 /*
  * attn_selftest_exp2 -- evaluates, on the device, the polynomial 2^x that

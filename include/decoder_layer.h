@@ -33,14 +33,17 @@
  * Sizes: B, S >= 1; hidden and inter multiples of 8; Hq % Hkv == 0; D 64 or
  * 128; eps >= 0; rope_theta > 1 (LLaMA3: eps 1e-5, theta 500000).
  *
- * The GEMMs are cuBLAS calls (fp16 in, fp32 accumulation, fp16 out; the
- * residual adds ride in their epilogues as beta = 1); RMSNorm, RoPE with the
- * head split, the head merge and SwiGLU are this library's sm_100a kernels,
- * and the attention is attn_fwd.  Each call launches them in order on
- * `stream`; the library keeps one cuBLAS handle per (device, stream), created
- * on first use and kept until the process exits, and the attention's redo
- * list as attn_fwd does.  Calls that share a stream must not be issued from
- * two host threads at once.
+ * The GEMMs are this library's tcgen05 kernel (2-SM tensor-core tiles of
+ * 256 x 256, fp16 in, fp32 accumulation), with the element steps fused into
+ * their epilogues: RoPE and the head split into the QKV projection, SwiGLU
+ * into the gate/up projection, the residual adds into the O and down
+ * projections; the O projection reads the attention output head-major when
+ * S % 128 == 0 (otherwise a head-merge kernel runs first).  Each fused step
+ * rounds where the unfused layer stores a tensor, so the stored values are
+ * those of the sequence above.  RMSNorm is a separate kernel and the
+ * attention is attn_fwd.  Each call launches them in order on `stream`.
+ * Their bounded waits report into the stream's status block, like
+ * attn_fwd's (read with attn_device_status()).
  */
 #ifndef ATTN_B200_DECODER_LAYER_H
 #define ATTN_B200_DECODER_LAYER_H
@@ -56,9 +59,9 @@ extern "C" {
 /*
  * attn_decoder_layer_workspace_bytes -- bytes of device workspace that
  * attn_decoder_layer_fwd needs for these sizes (all intermediates: the rotary
- * table, RMSNorm outputs, the QKV and gate/up products, Q/K/V/O head-major,
- * LSE, the residual stream h and the SwiGLU output; each region rounded up to
- * 256 bytes).  Returns 0 for sizes attn_decoder_layer_fwd rejects.
+ * table, RMSNorm outputs, Q/K/V/O head-major, LSE, the residual stream h and
+ * the SwiGLU output; each region rounded up to 256 bytes).  Returns 0 for
+ * sizes attn_decoder_layer_fwd rejects.
  */
 size_t attn_decoder_layer_workspace_bytes(int B, int S, int hidden, int Hq, int Hkv, int D,
                                           int inter);
@@ -74,11 +77,11 @@ size_t attn_decoder_layer_workspace_bytes(int B, int S, int hidden, int Hq, int 
  *   stream : cudaStream_t to launch on (asynchronous).
  * Returns ATTN_OK once everything is enqueued; ATTN_ERR_NULL, ATTN_ERR_SHAPE
  * (sizes, eps, theta), ATTN_ERR_UNSUPPORTED (D), ATTN_ERR_ALIGN,
- * ATTN_ERR_WORKSPACE before launching anything; ATTN_ERR_CUDA when a launch or
- * a cuBLAS call fails; the attention's status otherwise.  After a failure past
- * validation, earlier steps may already be enqueued: y and the workspace are
- * then undefined.  A timed-out wait in the attention is reported by
- * attn_device_status().
+ * ATTN_ERR_WORKSPACE before launching anything; ATTN_ERR_CUDA when a launch
+ * fails; the attention's status otherwise.  After a failure past validation,
+ * earlier steps may already be enqueued: y and the workspace are then
+ * undefined.  A timed-out wait in any of the kernels is reported by
+ * attn_device_status() on `stream`.
  */
 attn_status attn_decoder_layer_fwd(const void* x, const void* w_attn_norm, const void* w_qkv,
                                    const void* w_o, const void* w_mlp_norm, const void* w_gate_up,

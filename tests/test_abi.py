@@ -37,7 +37,7 @@ def test_exports_every_declared_symbol(lib):
 
 
 def test_version_and_strings(lib):
-    assert attn.version() >> 16 == 1
+    assert attn.version() >> 16 == 2
     for code in range(8):
         s = attn.status_string(code)
         assert s.startswith(attn.STATUS_NAMES[code])
@@ -58,8 +58,9 @@ def test_validation_before_launch(lib):
     assert call(lib, Hkv=3) == SHAPE          # Hq % Hkv != 0
     assert call(lib, Hq=0) == SHAPE
     assert call(lib, D=96) == UNSUP
-    assert call(lib, D=256) == UNSUP
-    assert call(lib, B=65536, Hq=1, Hkv=1, S=128) == SHAPE
+    assert call(lib, D=192) == UNSUP
+    assert call(lib, D=512) == UNSUP
+    assert call(lib, B=65536, Hq=1, Hkv=1, S=32768) == SHAPE  # key rows overflow 2^31
     assert call(lib, B=64, Hq=64, Hkv=8, S=1 << 20) == SHAPE  # row index overflow
     assert call(lib, q=FAKE + 8) == ALIGN
     assert call(lib, lse=FAKE + 2) == ALIGN

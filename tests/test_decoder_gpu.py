@@ -89,6 +89,14 @@ def test_decoder_llama3_8b_dims():
     _check(x, w, y, m["Hq"], m["Hkv"], m["D"], "llama3-8b dims, S=130")
 
 
+def test_decoder_llama3_8b_dims_aligned():
+    """The full LLaMA3-8B dimensions with S a multiple of 128: the output
+    projection reads the attention output head-major (no merge step)."""
+    m = DECODER_MODELS["llama3-8b"]
+    x, w, y = _run(2, 256, m["hidden"], m["Hq"], m["Hkv"], m["D"], m["inter"], seed=69)
+    _check(x, w, y, m["Hq"], m["Hkv"], m["D"], "llama3-8b dims, B=2 S=256")
+
+
 def test_decoder_in_place_and_deterministic():
     B, S, hidden, Hq, Hkv, D, inter = 2, 256, 256, 4, 2, 128, 512
     x, w, y = _run(B, S, hidden, Hq, Hkv, D, inter, seed=71)

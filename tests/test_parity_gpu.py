@@ -102,6 +102,56 @@ def test_d64_sampled(causal):
     parity.sampled_check(q, k, v, o, lse, causal, n_random=512, seed=31)
 
 
+# head dimension 256: one 128-row tile per work item, 64-key blocks, S
+# double-buffered in TMEM
+D256 = [(1, 2, 1, 64), (1, 4, 2, 384), (2, 4, 2, 200), (1, 6, 3, 1000), (1, 2, 2, 1)]
+
+
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("B,Hq,Hkv,S", D256)
+def test_d256_full(B, Hq, Hkv, S, causal):
+    parity.full_check(B, Hq, Hkv, S, 256, causal, seed=61)
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_d256_stress_full(causal):
+    parity.full_check(1, 8, 2, 700, 256, causal, seed=63, qk_std=4.0)
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_d256_large_outputs(causal):
+    """Every row with |O| >= 4: every item goes through the exact pass."""
+    B, Hq, Hkv, S, D = 1, 4, 2, 640, 256
+    q, k, _ = make_qkv(B, Hq, Hkv, S, D, seed=65, qk_std=4.0, device="cuda")
+    v = _large_v(B, Hkv, S, D, 66)
+    attn.device_status_ex()
+    o, lse = parity.run_gpu(q, k, v, causal)
+    import oracle
+    o_ref, lse_ref = oracle.attention(q.cpu().double().numpy(), k.cpu().double().numpy(),
+                                      v.cpu().double().numpy(), causal)
+    parity.assert_close(o.cpu().double().numpy(), o_ref, lse.cpu().double().numpy(), lse_ref,
+                        "D256 large V causal=%d" % causal)
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_d256_qk(causal):
+    q, k, v = _qk_inputs(1, 4, 2, 200, 450, 256, seed=67)
+    _qk_check(q, k, v, causal, "D256 Sq200 Sk450")
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_d256_sampled(causal):
+    q, k, v = make_qkv(4, 16, 4, 4096, 256, seed=69, device="cuda")
+    o, lse = parity.run_gpu(q, k, v, causal)
+    parity.sampled_check(q, k, v, o, lse, causal, n_random=256, seed=69)
+
+
+@pytest.mark.parametrize("variant", [1, 2, 4, 15])
+def test_d256_variants(variant):
+    q, k, v = make_qkv(1, 8, 2, 520, 256, seed=71, qk_std=4.0, device="cuda")
+    _variant_check(q, k, v, True, variant, "D256 %s" % attn.variant_name(variant))
+
+
 # Sq query rows over Sk keys (attn_fwd_qk); causal windows aligned bottom-right
 QK = [(1, 4, 2, 1, 513), (2, 4, 2, 77, 300), (1, 8, 2, 128, 1000), (1, 6, 3, 257, 1024),
       (2, 4, 1, 300, 300)]
@@ -199,10 +249,10 @@ def test_deterministic():
 
 
 def test_concurrent_streams():
-    """Calls on two streams run at the same time, each with its own redo list:
-    large-V inputs (every item listed for the redo pass) on one stream and
-    N(0,1) inputs on the other give the same bytes as the same calls made one
-    after another on the default stream."""
+    """Calls on two streams run at the same time, each with its own status
+    block: large-V inputs (every item recomputed by the exact pass) on one
+    stream and N(0,1) inputs on the other give the same bytes as the same
+    calls made one after another on the default stream."""
     B, Hq, Hkv, S, D = 2, 8, 2, 640, 128
     qa, ka, _ = make_qkv(B, Hq, Hkv, S, D, seed=71, device="cuda")
     va = _large_v(B, Hkv, S, D, seed=73)
@@ -309,16 +359,84 @@ def test_large_outputs_exact_rows(causal):
                         "large V causal=%d" % causal)
 
 
-def test_large_outputs_overflow_scan():
-    """More flagged rows than the list holds (2^16): the fixup kernel scans O
-    itself.  Sampled rows against the oracle."""
-    B, Hq, Hkv, S, D = 4, 16, 4, 2048, 128   # 131072 rows, all flagged
+def test_large_outputs_every_item_exact():
+    """Every 256-row item of every CTA is marked (many per CTA): the exact
+    pass recomputes all of them in the same launch.  Sampled rows against the
+    oracle, and the call's status block counts every item."""
+    B, Hq, Hkv, S, D = 4, 16, 4, 2048, 128   # 512 items of 256 rows, all marked
     q, k, _ = make_qkv(B, Hq, Hkv, S, D, seed=23, qk_std=4.0, device="cuda")
     v = _large_v(B, Hkv, S, D, 24)
-    o, lse = parity.run_gpu(q, k, v, True)
+    attn.device_status_ex()  # clear
+    o = torch.full_like(q, float("nan"))
+    lse = torch.full((B, Hq, S), float("nan"), dtype=torch.float32, device="cuda")
+    attn.attn_fwd(q, k, v, True, o=o, lse=lse)
+    st, site, n_exact = attn.device_status_ex()
+    assert st == attn.ATTN_OK, "device status %d at site %#x" % (st, site)
+    assert n_exact == B * Hq * (S // 256), n_exact
     parity.sampled_check(q, k, v, o, lse, True, n_random=512, seed=25, full_heads=True)
-    # the list is empty again: a plain call right after still passes
+    # nothing carries over: a plain call right after still passes
     parity.full_check(1, 2, 1, 256, 128, True, seed=26)
+
+
+def test_exact_pass_only_where_needed():
+    """N(0,1) inputs at a long sequence: outputs average many V rows, so only
+    the first rows of a head can reach |O| >= 3.98 -- few items, all of them
+    in the last row block of the walk order (row block 0 of each head)."""
+    B, Hq, Hkv, S, D = 2, 16, 4, 4096, 128
+    q, k, v = make_qkv(B, Hq, Hkv, S, D, seed=27, device="cuda")
+    attn.device_status_ex()
+    o, lse = attn.attn_fwd(q, k, v, True)
+    st, site, n_exact = attn.device_status_ex()
+    assert st == attn.ATTN_OK, "device status %d at site %#x" % (st, site)
+    assert n_exact <= B * Hq, n_exact
+    parity.sampled_check(q, k, v, o, lse, True, n_random=256, seed=27, full_heads=False)
+
+
+def test_status_blocks_are_per_stream():
+    """A wait that runs out on one stream is reported by that stream's status
+    and not by another stream's, even while that other stream runs attention."""
+    s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
+    q, k, v = make_qkv(1, 8, 2, 1024, 128, seed=31, device="cuda")
+    assert attn.selftest_wait_timeout(20_000_000, stream=s1) == attn.ATTN_ERR_DEVICE_TIMEOUT
+    with torch.cuda.stream(s2):
+        attn.attn_fwd(q, k, v, True, stream=s2)
+    assert attn.device_status(s2) == (attn.ATTN_OK, 0)
+    # the self-test read (and cleared) s1's block itself; nothing is left there
+    assert attn.device_status(s1) == (attn.ATTN_OK, 0)
+
+
+# Items of two 128-row tiles (the launch has at least as many 256-row items as
+# SMs): full oracle checks, including an odd number of row blocks (the last
+# item has tile A only) and a ragged last tile.
+TWO_TILE = [(2, 40, 8, 512, 128, 1.0), (1, 64, 8, 600, 128, 1.0), (1, 64, 8, 700, 128, 4.0),
+            (1, 80, 8, 520, 64, 1.0)]
+
+
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("B,Hq,Hkv,S,D,qk_std", TWO_TILE)
+def test_two_tile_items_full(B, Hq, Hkv, S, D, qk_std, causal):
+    parity.full_check(B, Hq, Hkv, S, D, causal, seed=33, qk_std=qk_std)
+
+
+def test_call_split_into_launches():
+    """More items than one launch's per-CTA marks hold (2048 per CTA): the
+    call runs as several launches over batch ranges.  Sampled rows from the
+    first and the last batch elements."""
+    B, Hq, Hkv, S, D = 2500, 64, 8, 300, 64   # 320000 items of 256 rows
+    q, k, v = make_qkv(B, Hq, Hkv, S, D, seed=35, device="cuda")
+    o, lse = parity.run_gpu(q, k, v, True)
+    import oracle
+    for b in (0, 1, B // 2, B - 2, B - 1):
+        for hq in (0, Hq - 1):
+            o_ref, lse_ref = oracle.attention(q[b:b + 1, hq:hq + 1].cpu().double().numpy(),
+                                              k[b:b + 1, hq // 8:hq // 8 + 1].cpu().double().numpy(),
+                                              v[b:b + 1, hq // 8:hq // 8 + 1].cpu().double().numpy(),
+                                              True)
+            parity.assert_close(o[b:b + 1, hq:hq + 1].cpu().double().numpy(), o_ref,
+                                lse[b:b + 1, hq:hq + 1].cpu().double().numpy(), lse_ref,
+                                "split call b=%d hq=%d" % (b, hq))
+    del q, k, v, o, lse
+    torch.cuda.empty_cache()
 
 
 def test_fma_pipe_exp2_error_bound():
@@ -340,11 +458,13 @@ def test_fma_pipe_exp2_error_bound():
     assert torch.all(lo >= 0) and torch.all(lo < 2.0 ** -124), lo
 
 
-# Every fused-pass variant (0..4 of every 8 exponential pairs from the FMA-pipe
-# polynomial) through attn_fwd_variant, against the oracle: both head dims, a
-# ragged tail, logits of standard deviation 1 and 16.
+# Every fused-kernel variant (two-tile ping-pong with one or two MMA-issuing
+# warps, one tile with S double-buffered and one or two softmax warps per lane
+# quadrant, x 0..4 of every 8 exponential pairs from the FMA-pipe polynomial)
+# through attn_fwd_variant, against the oracle: both head dims, a ragged
+# tail, logits of standard deviation 1 and 16, one-tile and two-tile items.
 VARIANT_CASES = [(2, 4, 2, 383, 128, 1.0), (1, 8, 2, 512, 128, 4.0), (2, 4, 2, 329, 64, 1.0),
-                 (1, 4, 2, 640, 64, 4.0)]
+                 (1, 4, 2, 640, 64, 4.0), (1, 64, 8, 700, 128, 1.0)]
 
 
 def _variant_check(q, k, v, causal, variant, what):
@@ -359,19 +479,19 @@ def _variant_check(q, k, v, causal, variant, what):
                         what)
 
 
-@pytest.mark.parametrize("variant", range(5))
+@pytest.mark.parametrize("variant", range(20))
 @pytest.mark.parametrize("causal", [True, False])
 @pytest.mark.parametrize("B,Hq,Hkv,S,D,qk_std", VARIANT_CASES)
 def test_variant_full(B, Hq, Hkv, S, D, qk_std, causal, variant):
-    assert attn.variant_count() == 5
+    assert attn.variant_count() == 20
     q, k, v = make_qkv(B, Hq, Hkv, S, D, seed=41, qk_std=qk_std, device="cuda")
     _variant_check(q, k, v, causal, variant, "%s B%d Hq%d S%d D%d std%g causal=%d" % (
         attn.variant_name(variant), B, Hq, S, D, qk_std, causal))
 
 
-@pytest.mark.parametrize("variant", [2, 4])
+@pytest.mark.parametrize("variant", [2, 4, 5, 7, 10, 12, 15, 17])
 def test_variant_large_outputs(variant):
-    """Large V: every item goes through the redo pass after an emulating fused pass."""
+    """Large V: every item goes through the exact pass after an emulating fast pass."""
     q, k, _ = make_qkv(1, 8, 2, 384, 128, seed=43, device="cuda")
     v = _large_v(1, 2, 384, 128, seed=47)
     _variant_check(q, k, v, True, variant, "large V, %s" % attn.variant_name(variant))

@@ -40,9 +40,11 @@ def expected_variant(rules, D, causal, Sk):
 
 def test_count_and_names(lib):
     n = attn.variant_count()
-    assert n == 5
+    assert n == 20
     names = [attn.variant_name(i) for i in range(n)]
-    assert names == ["fma_exp2_pairs=%d/8" % i for i in range(5)]
+    structures = ["pingpong,mma_issuers=1", "pingpong,mma_issuers=2", "dbuf,softmax_split=1",
+                  "dbuf,softmax_split=2"]
+    assert names == ["%s,fma_exp2_pairs=%d/8" % (structures[i // 5], i % 5) for i in range(20)]
     assert attn.variant_name(-1) is None and attn.variant_name(n) is None
 
 
