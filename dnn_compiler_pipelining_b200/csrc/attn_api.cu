@@ -45,10 +45,11 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 // ---------------------------------------------------------------------------
 // fused-kernel variants: a pipeline structure x kEmu FMA-pipe exponentials
-// per 8 column pairs.  Structures: 0 two-tile ping-pong, one MMA-issuing
-// warp; 1 the same with one issuing warp per tile; 2 one tile with S
-// double-buffered in TMEM; 3 the same with two softmax warps per lane
-// quadrant.  Head dimension 256 has only the double-buffered kernel with one
+// per 8 column pairs.  Structures: 0 two-tile ping-pong, the tiles two row
+// blocks of one head; 1 the same kernel with the tiles the same rows of two
+// query heads of one kv group (when the group has an even number of heads;
+// else as 0); 2 one tile with S double-buffered in TMEM; 3 the same with two
+// softmax warps per lane quadrant.  Head dimension 256 has only the double-buffered kernel with one
 // softmax warp per quadrant (shared memory has no room for more): every
 // structure maps to it there.
 // ---------------------------------------------------------------------------
@@ -63,8 +64,9 @@ using FwdKernel = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorM
 struct KernelChoice {
   FwdKernel fn;
   size_t smem;
-  int one_tile;  // items are one 128-row tile
-  int kv_box;    // rows of a K / V tile
+  int one_tile;    // items are one 128-row tile
+  int kv_box;      // rows of a K / V tile
+  int pair_heads;  // two-tile items pair query heads
 };
 
 template <int kD, int kV>
@@ -72,12 +74,12 @@ KernelChoice kernel_choice_v() {
   constexpr int s = variant_structure(kV), e = variant_emu(kV);
   if constexpr (kD == 256) {
     return {&db::attn_fwd_db_kernel<256, 1, e>, sizeof(db::SharedDb<256, 1>), 1,
-            db::Cfg<256>::kBN};
+            db::Cfg<256>::kBN, 0};
   } else if constexpr (s == 0 || s == 1) {
-    return {&attn_fwd_kernel<kD, e, s + 1>, sizeof(SharedFwdT<kD>), 0, kBlockN};
+    return {&attn_fwd_kernel<kD, e>, sizeof(SharedFwdT<kD>), 0, kBlockN, s == 1};
   } else {
     return {&db::attn_fwd_db_kernel<kD, s - 1, e>, sizeof(db::SharedDb<kD, s - 1>), 1,
-            db::Cfg<kD>::kBN};
+            db::Cfg<kD>::kBN, 0};
   }
 }
 template <int kD, int... kV>
@@ -247,7 +249,8 @@ size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 // Kernel parameters of one launch over B batch elements (Sq query rows over
 // Sk keys) on a device with `sms` SMs and `l2` bytes of L2.
 FwdParams make_params(void* o, float* lse, unsigned int* status, int B, int Hq, int Hkv, int Sq,
-                      int Sk, int D, int causal, int sms, int l2, bool one_tile) {
+                      int Sk, int D, int causal, int sms, int l2, bool one_tile,
+                      bool pair_heads) {
   FwdParams p;
   p.o = static_cast<__half*>(o);
   p.lse = lse;
@@ -266,8 +269,9 @@ FwdParams make_params(void* o, float* lse, unsigned int* status, int B, int Hq, 
   // one tile per item, or two-tile items would leave SMs idle
   const long long heads = static_cast<long long>(B) * Hq;
   p.item_tiles = (one_tile || heads * ((p.n_qb + 1) / 2) < sms) ? 1 : 2;
-  p.n_qi = (p.n_qb + p.item_tiles - 1) / p.item_tiles;
-  p.n_items = static_cast<int>(heads * p.n_qi);
+  p.pair_heads = (pair_heads && p.item_tiles == 2 && p.group % 2 == 0) ? 1 : 0;
+  p.n_qi = p.pair_heads ? p.n_qb : (p.n_qb + p.item_tiles - 1) / p.item_tiles;
+  p.n_items = static_cast<int>(heads / (1 + p.pair_heads) * p.n_qi);
   // Longest first (snake) balances a causal launch; it walks all kv heads at
   // once, so it is used only when all of K and V stay resident in L2.
   const double kv_bytes = 2.0 * B * Hkv * static_cast<double>(Sk) * D * 2;
@@ -285,7 +289,7 @@ attn_status launch_call(const void* q, const void* k, const void* v, void* o, fl
   const int sms = g_dev_sms[dev];
   const KernelChoice& kc = kernel_choice(D, variant);
   const FwdParams whole = make_params(o, lse, status, B, Hq, Hkv, Sq, Sk, D, causal, sms,
-                                      g_dev_l2[dev], kc.one_tile != 0);
+                                      g_dev_l2[dev], kc.one_tile != 0, kc.pair_heads != 0);
   const long long per_b = static_cast<long long>(whole.n_items) / B;
   const long long max_items = static_cast<long long>(sms) * kMaxItemsPerCta;
   const int chunk_b = static_cast<int>(per_b >= max_items ? 1 : max_items / per_b);
@@ -307,7 +311,7 @@ attn_status launch_call(const void* q, const void* k, const void* v, void* o, fl
         !encode_rows_map(&tv, vc, static_cast<uint64_t>(nb) * Hkv * Sk, D, kv_box))
       return ATTN_ERR_CUDA;
     const FwdParams p = make_params(oc, lc, status, nb, Hq, Hkv, Sq, Sk, D, causal, sms,
-                                    g_dev_l2[dev], kc.one_tile != 0);
+                                    g_dev_l2[dev], kc.one_tile != 0, kc.pair_heads != 0);
     const int grid = p.n_items < sms ? p.n_items : sms;
     kc.fn<<<grid, kThreads, kc.smem, cs>>>(tq, tk, tv, p);
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
@@ -425,7 +429,7 @@ const char* attn_variant_name(int variant) {
   static std::once_flag once;
   std::call_once(once, [] {
     static const char* kStructureNames[kStructures] = {
-        "pingpong,mma_issuers=1", "pingpong,mma_issuers=2", "dbuf,softmax_split=1",
+        "pingpong,row_pairs", "pingpong,head_pairs", "dbuf,softmax_split=1",
         "dbuf,softmax_split=2"};
     for (int v = 0; v < kNumVariants; ++v)
       std::snprintf(names[v], sizeof(names[v]), "%s,fma_exp2_pairs=%d/8",

@@ -222,7 +222,9 @@ __device__ __forceinline__ void producer(Sm* sm, const FwdParams& p,
 
 // MMA issuer (whole warp).  Per item of n blocks, step t = 0..n+1 issues
 // PV(t-2) (t >= 2) and then S(t) (t < n); g0 + t is the CTA-wide block
-// index that picks the S buffer.
+// index that picks the S buffer.  One thread issues every MMA: S(t)
+// overwrites the columns PV(t-2) reads and every PV accumulates into O, and
+// only MMAs of one thread are ordered by the pipe.
 template <int kD, class Sm>
 __device__ __forceinline__ void mma(Sm* sm, const FwdParams& p, uint32_t tmem,
                                     volatile int* abort) {
@@ -279,167 +281,173 @@ __device__ __forceinline__ void mma(Sm* sm, const FwdParams& p, uint32_t tmem,
   drain_wait(smem_addr(&sm->drain), 0, to, p.status);
 }
 
-// Softmax warp: TMEM lane quadrant q = warp % 4 (rows 32 q ..), column half
-// h = warp / 4 of each key block (kSplit = 2) or all of it (kSplit = 1).
-template <int kD, int kSplit, int kEmu>
-__device__ __forceinline__ void softmax(SharedDb<kD, kSplit>* sm, const FwdParams& p, uint32_t tmem,
-                                        int warp, int lane, volatile int* abort) {
+// The key blocks of one item for one softmax warp: TMEM lane quadrant
+// `quad` (rows 32 quad ..), column half h of each key block (kSplit = 2) or
+// all of it (kSplit = 1).  kHilo: the exact pass.  Returns false if a wait
+// gave up; m_use and l hold the row's statistics (l: this half's) on return.
+template <int kD, int kSplit, int kEmu, bool kHilo>
+__device__ __forceinline__ bool softmax_item(SharedDb<kD, kSplit>* sm, const FwdParams& p,
+                                             uint32_t lane_base, int quad, int h, int r, int lane,
+                                             int n, int key_lim, int j_mask, int& g, float& m_use,
+                                             float& l, volatile int* abort) {
   using C = Cfg<kD>;
   constexpr int kCols = C::kBN / kSplit;  // keys of a block this warp handles
   const uint64_t to = p.timeout_ns;
+  const uint32_t o_t = lane_base + C::kTmemO + h * (kD / kSplit);
+  const float sc = p.scale_log2;
+  m_use = -INFINITY;
+  l = 0.f;
+  for (int j = 0; j < n; ++j, ++g) {
+    const int b = g & 1;
+    const uint32_t s_t = lane_base + tmem_s(b, C::kBN);
+    bool ok = mbar_wait(smem_addr(&sm->s_full[b]), (g >> 1) & 1, abort, to, p.status,
+                        kSiteSoftmaxS);
+    if (!__all_sync(0xffffffffu, ok)) return false;
+    tc_fence_after();
+    uint32_t u[kCols];
+#pragma unroll
+    for (int c = 0; c < kCols; c += 32) tmem_ld32(s_t + h * kCols + c, &u[c]);
+    tmem_wait_ld();
+#pragma unroll
+    for (int c = 0; c < kCols; c += 32) reg_dep32(&u[c]);
+    if (j >= j_mask) {
+      const int lim = key_lim - j * C::kBN - h * kCols;
+#pragma unroll
+      for (int c = 0; c < kCols; ++c)
+        if (c > lim) u[c] = 0xff800000u;  // -inf
+    }
+    float mx8[8];
+#pragma unroll
+    for (int t = 0; t < 8; ++t) mx8[t] = fmaxf(__uint_as_float(u[t]), __uint_as_float(u[8 + t]));
+#pragma unroll
+    for (int c = 16; c + 16 <= kCols; c += 16)
+#pragma unroll
+      for (int t = 0; t < 8; ++t)
+        mx8[t] = fmax3(mx8[t], __uint_as_float(u[c + t]), __uint_as_float(u[c + 8 + t]));
+    float cand = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
+                       fmaxf(mx8[6], mx8[7]));
+    if constexpr (kSplit == 2) {
+      // the partner warp (same rows, other half of the keys) posts its
+      // partial maximum too; xmax[block parity][quad] completes when both
+      // have.  A slot is written again two blocks later, after the partner
+      // passed the next block's exchange and so read this one.
+      sm->red_max[g & 1][h][r] = cand;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_addr(&sm->xmax[g & 1][quad]));
+      ok = mbar_wait<true>(smem_addr(&sm->xmax[g & 1][quad]), (g >> 1) & 1, abort, to, p.status,
+                           kSiteSoftmaxStats);
+      if (!__all_sync(0xffffffffu, ok)) return false;
+      cand = fmaxf(cand, sm->red_max[g & 1][h ^ 1][r]);
+    }
+    cand *= sc;
+    if (j == 0) {
+      m_use = cand;
+    } else {
+      const bool grow = cand > m_use + kRescaleLog2;
+      if (__any_sync(0xffffffffu, grow)) {
+        // O must hold PV(g-1) before it is rescaled
+        ok = mbar_wait(smem_addr(&sm->pv_done), (g - 1) & 1, abort, to, p.status, kSiteSoftmaxS);
+        if (!__all_sync(0xffffffffu, ok)) return false;
+        tc_fence_after();
+        const float alpha = grow ? ex2_approx(m_use - cand) : 1.0f;
+#pragma unroll 1
+        for (int c = 0; c < kD / kSplit; c += 32) {
+          uint32_t wv[32];
+          tmem_ld32(o_t + c, wv);
+          tmem_wait_ld();
+          reg_dep32(wv);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) wv[i] = __float_as_uint(__uint_as_float(wv[i]) * alpha);
+          tmem_st32(o_t + c, wv);
+        }
+        if (grow) {
+          l *= alpha;
+          m_use = cand;
+        }
+      }
+    }
+    const float neg_m = -m_use;
+    float lp[4] = {0.f, 0.f, 0.f, 0.f};
+    // this warp's keys go to P columns [h kCols / 2, (h + 1) kCols / 2)
+    const uint32_t p_t = s_t + h * (kCols / 2);
+    if constexpr (!kHilo) {
+      const float2 sc2 = make_float2(sc, sc);
+      const float2 nm2 = make_float2(neg_m, neg_m);
+#pragma unroll
+      for (int c = 0; c < kCols / 16; ++c) {
+        uint32_t ph[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float2 s2 = make_float2(__uint_as_float(u[c * 16 + 2 * i]),
+                                        __uint_as_float(u[c * 16 + 2 * i + 1]));
+          const float2 x2 = __ffma2_rn(s2, sc2, nm2);
+          float2 p2;
+          if (i < kEmu) {
+            p2 = exp2_poly2(x2);
+          } else {
+            p2.x = ex2_approx(x2.x);
+            p2.y = ex2_approx(x2.y);
+          }
+          ph[i] = pack_half2(p2.x, p2.y);
+          lp[i & 3] = add_half2_f32(ph[i], lp[i & 3]);
+        }
+        tmem_st8(p_t + c * 8, ph);
+      }
+    } else {
+      // P = hi + lo: hi over P's columns, lo kBN / 2 columns further
+#pragma unroll
+      for (int c = 0; c < kCols / 16; ++c) {
+        uint32_t ph[8], pl[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float p0 = ex2_approx(fmaf(__uint_as_float(u[c * 16 + 2 * i]), sc, neg_m));
+          const float p1 = ex2_approx(fmaf(__uint_as_float(u[c * 16 + 2 * i + 1]), sc, neg_m));
+          ph[i] = pack_half2(p0, p1);
+          const float2 hh = __half22float2(*reinterpret_cast<const __half2*>(&ph[i]));
+          pl[i] = pack_half2(p0 - hh.x, p1 - hh.y);
+          lp[i & 3] += p0 + p1;
+        }
+        tmem_st8(p_t + c * 8, ph);
+        tmem_st8(p_t + C::kBN / 2 + c * 8, pl);
+      }
+    }
+    l += (lp[0] + lp[1]) + (lp[2] + lp[3]);
+    tmem_wait_st();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(smem_addr(&sm->p_full[b]));
+  }
+  return true;
+}
+
+template <int kD, int kSplit, int kEmu>
+__device__ __forceinline__ void softmax(SharedDb<kD, kSplit>* sm, const FwdParams& p,
+                                        uint32_t tmem, int warp, int lane, volatile int* abort) {
+  using C = Cfg<kD>;
   const int quad = warp & 3;
   const int h = kSplit == 2 ? (warp >> 2) : 0;
   const int r = quad * 32 + lane;
   const uint32_t lane_base = tmem + (static_cast<uint32_t>(quad * 32) << 16);
-  const uint32_t o_t = lane_base + C::kTmemO + h * (kD / kSplit);
-  const float sc = p.scale_log2;
   int g = 0;      // key blocks so far (all items)
   int acnt = 0;   // items so far
   bool ok = true;
   ItemWalk w;
   int item;
   while (ok && (item = walk(w, p, sm, abort, ok, kSiteSoftmaxRedo)) >= 0) {
-    const bool hilo = w.exact;
     const Item it = decode_item(p, item);
     const int n = n_blocks<C::kBN>(p, it);
     const int i_row = it.qb0 * kBlockM + r;
     const int key_lim = p.causal ? min(i_row + p.off, p.Sk - 1) : p.Sk - 1;
     // the first block in which some lane of the warp has keys to mask
     const int j_mask = (__shfl_sync(0xffffffffu, key_lim, 0) + 1) / C::kBN;
-    float m_use = -INFINITY;
-    float l = 0.f;
-    for (int j = 0; j < n; ++j, ++g) {
-      const int b = g & 1;
-      const uint32_t s_t = lane_base + tmem_s(b, C::kBN);
-      ok = mbar_wait(smem_addr(&sm->s_full[b]), (g >> 1) & 1, abort, to, p.status, kSiteSoftmaxS);
-      if (!__all_sync(0xffffffffu, ok)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      uint32_t u[kCols];
-#pragma unroll
-      for (int c = 0; c < kCols; c += 32) tmem_ld32(s_t + h * kCols + c, &u[c]);
-      tmem_wait_ld();
-#pragma unroll
-      for (int c = 0; c < kCols; c += 32) reg_dep32(&u[c]);
-      if (j >= j_mask) {
-        const int lim = key_lim - j * C::kBN - h * kCols;
-#pragma unroll
-        for (int c = 0; c < kCols; ++c)
-          if (c > lim) u[c] = 0xff800000u;  // -inf
-      }
-      float mx8[8];
-#pragma unroll
-      for (int t = 0; t < 8; ++t) mx8[t] = fmaxf(__uint_as_float(u[t]), __uint_as_float(u[8 + t]));
-#pragma unroll
-      for (int c = 16; c + 16 <= kCols; c += 16)
-#pragma unroll
-        for (int t = 0; t < 8; ++t)
-          mx8[t] = fmax3(mx8[t], __uint_as_float(u[c + t]), __uint_as_float(u[c + 8 + t]));
-      float cand = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
-                         fmaxf(mx8[6], mx8[7]));
-      if constexpr (kSplit == 2) {
-        // the partner warp (same rows, other half of the keys) posts its
-        // partial maximum too; xmax[block parity][quad] completes when both
-        // have.  A slot is written again two blocks later, after the partner
-        // passed the next block's exchange and so read this one.
-        sm->red_max[g & 1][h][r] = cand;
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_addr(&sm->xmax[g & 1][quad]));
-        ok = mbar_wait<true>(smem_addr(&sm->xmax[g & 1][quad]), (g >> 1) & 1, abort, to, p.status,
-                             kSiteSoftmaxStats);
-        if (!__all_sync(0xffffffffu, ok)) {
-          ok = false;
-          break;
-        }
-        cand = fmaxf(cand, sm->red_max[g & 1][h ^ 1][r]);
-      }
-      cand *= sc;
-      if (j == 0) {
-        m_use = cand;
-      } else {
-        const bool grow = cand > m_use + kRescaleLog2;
-        if (__any_sync(0xffffffffu, grow)) {
-          // O must hold PV(g-1) before it is rescaled
-          ok = mbar_wait(smem_addr(&sm->pv_done), (g - 1) & 1, abort, to, p.status,
-                         kSiteSoftmaxS);
-          if (!__all_sync(0xffffffffu, ok)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const float alpha = grow ? ex2_approx(m_use - cand) : 1.0f;
-#pragma unroll 1
-          for (int c = 0; c < kD / kSplit; c += 32) {
-            uint32_t wv[32];
-            tmem_ld32(o_t + c, wv);
-            tmem_wait_ld();
-            reg_dep32(wv);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) wv[i] = __float_as_uint(__uint_as_float(wv[i]) * alpha);
-            tmem_st32(o_t + c, wv);
-          }
-          if (grow) {
-            l *= alpha;
-            m_use = cand;
-          }
-        }
-      }
-      const float neg_m = -m_use;
-      float lp[4] = {0.f, 0.f, 0.f, 0.f};
-      // this warp's keys go to P columns [h kCols / 2, (h + 1) kCols / 2)
-      const uint32_t p_t = s_t + h * (kCols / 2);
-      if (!hilo) {
-        const float2 sc2 = make_float2(sc, sc);
-        const float2 nm2 = make_float2(neg_m, neg_m);
-#pragma unroll
-        for (int c = 0; c < kCols / 16; ++c) {
-          uint32_t ph[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const float2 s2 = make_float2(__uint_as_float(u[c * 16 + 2 * i]),
-                                          __uint_as_float(u[c * 16 + 2 * i + 1]));
-            const float2 x2 = __ffma2_rn(s2, sc2, nm2);
-            float2 p2;
-            if (i < kEmu) {
-              p2 = exp2_poly2(x2);
-            } else {
-              p2.x = ex2_approx(x2.x);
-              p2.y = ex2_approx(x2.y);
-            }
-            ph[i] = pack_half2(p2.x, p2.y);
-            lp[i & 3] = add_half2_f32(ph[i], lp[i & 3]);
-          }
-          tmem_st8(p_t + c * 8, ph);
-        }
-      } else {
-        // P = hi + lo: hi over P's columns, lo kBN / 2 columns further
-#pragma unroll
-        for (int c = 0; c < kCols / 16; ++c) {
-          uint32_t ph[8], pl[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const float p0 = ex2_approx(fmaf(__uint_as_float(u[c * 16 + 2 * i]), sc, neg_m));
-            const float p1 = ex2_approx(fmaf(__uint_as_float(u[c * 16 + 2 * i + 1]), sc, neg_m));
-            ph[i] = pack_half2(p0, p1);
-            const float2 hh = __half22float2(*reinterpret_cast<const __half2*>(&ph[i]));
-            pl[i] = pack_half2(p0 - hh.x, p1 - hh.y);
-            lp[i & 3] += p0 + p1;
-          }
-          tmem_st8(p_t + c * 8, ph);
-          tmem_st8(p_t + C::kBN / 2 + c * 8, pl);
-        }
-      }
-      l += (lp[0] + lp[1]) + (lp[2] + lp[3]);
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_addr(&sm->p_full[b]));
-    }
+    float m_use, l;
+    ok = w.exact ? softmax_item<kD, kSplit, kEmu, true>(sm, p, lane_base, quad, h, r, lane, n,
+                                                         key_lim, j_mask, g, m_use, l, abort)
+                 : softmax_item<kD, kSplit, kEmu, false>(sm, p, lane_base, quad, h, r, lane, n,
+                                                          key_lim, j_mask, g, m_use, l, abort);
     if (!ok) break;
     ok = acnt == 0 ||
-         mbar_wait(smem_addr(&sm->stats_free), (acnt - 1) & 1, abort, to, p.status,
+         mbar_wait(smem_addr(&sm->stats_free), (acnt - 1) & 1, abort, p.timeout_ns, p.status,
                    kSiteSoftmaxStats);
     if (!__all_sync(0xffffffffu, ok)) {
       ok = false;

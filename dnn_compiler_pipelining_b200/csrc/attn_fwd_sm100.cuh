@@ -25,19 +25,20 @@
 //   warps 4-7   softmax of tile B
 //   warps 8-11  epilogue: O / l -> fp16, LSE, for both tiles
 //   warp 12     TMA producer of Q_A, Q_B (per item) and K_j (a ring)
-//   warp 13     MMA issuer: S_X = Q_X K_j^T, O_X += P_X V_j (both tiles, or
-//               tile A only when kIssuers == 2)
+//   warp 13     MMA issuer: S_X = Q_X K_j^T, O_X += P_X V_j (both tiles)
 //   warp 14     TMA producer of V_j (its own ring)
-//   warp 15     MMA issuer of tile B when kIssuers == 2, else idle
-// The MMA warps run whole: every lane takes the same branches and waits, and
-// one elected lane issues each MMA and commit.
+//   warp 15     idle
+// The MMA warp runs whole: every lane takes the same branches and waits, and
+// one elected lane issues each MMA and commit.  One thread issues every MMA:
+// a second issuing warp, even one taking strict turns with the first so that
+// the pipe sees the same order, measured 20% slower on B200.
 //
 // TMEM (512 columns): S_A [0,128), S_B [128,256), O_A [256,384),
 // O_B [384,512).  P_X (fp16) is written over the first 64 columns of S_X
 // (in the exact pass its low half over the next 64).
 //
-// Per tile X and key block j the issuer of X issues PV_X(j-1) and then
-// S_X(j); tcgen05 operations of one thread complete in order, so when S_X(j)
+// Per tile X and key block j the issuer issues PV_X(j-1) and then S_X(j);
+// tcgen05 operations of one thread complete in order, so when S_X(j)
 // signals s_full, O_X already holds P_X(j-1) V_{j-1} and the softmax may
 // rescale it, and P_X(j-1) has been read before S_X(j) overwrites it.
 //
@@ -104,8 +105,10 @@ struct FwdParams {
   int n_kb;              // ceil(Sk / 128) key blocks
   int group;             // Hq / Hkv
   int item_tiles;        // 2: items of two 128-row tiles; 1: one tile
-  int n_qi;              // items per (batch, head): ceil(n_qb / item_tiles)
-  int n_items;           // B * Hq * n_qi
+  int pair_heads;        // two-tile items: 1 = the same rows of two query heads of a kv
+                         // group, 0 = two consecutive row blocks of one head
+  int n_qi;              // items per (batch, head or head pair)
+  int n_items;
   int order;             // 0: kv-head major, round robin; 1: longest first, snake
   float scale_log2;      // log2(e) / sqrt(D)
   unsigned long long timeout_ns;
@@ -161,40 +164,46 @@ struct SharedFwdT {
 
 static_assert(sizeof(SharedFwdT<128>) <= 232448, "shared memory exceeds the 227 KiB per-block limit");
 
+// Tile x of an item is row block qb0 + x * dqb of query head hq + x * dhq.
 struct Item {
   int b, hq, g;
   int qb0;       // row block of tile A
+  int dqb, dhq;  // (1, 0): two row blocks of one head; (0, 1): two heads of one kv group
   int n_kv[2];   // key blocks of tile A, tile B (0: the tile is not part of the item)
   int n_blocks;  // max of the two
 };
 
 __device__ __forceinline__ Item decode_item(const FwdParams& p, int id) {
+  // the query heads (or head pairs) of a kv group an item can start at
+  const int members = p.pair_heads ? p.group / 2 : p.group;
   int qi, kvh, member;
   if (p.order == 0) {
     // kv-head major; inside a kv head: row blocks from last to first, the
     // group's query heads adjacent
-    const int per_kv = p.group * p.n_qi;
+    const int per_kv = members * p.n_qi;
     kvh = id / per_kv;
     const int rem = id - kvh * per_kv;
-    qi = p.n_qi - 1 - rem / p.group;
-    member = rem - (rem / p.group) * p.group;
+    qi = p.n_qi - 1 - rem / members;
+    member = rem - (rem / members) * members;
   } else {
     // row blocks from last (longest) to first; inside one, kv-head major
-    const int heads = p.B * p.Hq;
+    const int heads = p.B * p.Hkv * members;
     const int r = id / heads;
     const int rem = id - r * heads;
     qi = p.n_qi - 1 - r;
-    kvh = rem / p.group;
-    member = rem - kvh * p.group;
+    kvh = rem / members;
+    member = rem - kvh * members;
   }
   Item it;
   it.b = kvh / p.Hkv;
   it.g = kvh - it.b * p.Hkv;
-  it.hq = it.g * p.group + member;
-  it.qb0 = qi * p.item_tiles;
+  it.dhq = p.pair_heads;
+  it.dqb = p.pair_heads ? 0 : 1;
+  it.hq = it.g * p.group + member * (1 + p.pair_heads);
+  it.qb0 = p.pair_heads ? qi : qi * p.item_tiles;
 #pragma unroll
   for (int x = 0; x < 2; ++x) {
-    const int qb = it.qb0 + x;
+    const int qb = it.qb0 + x * it.dqb;
     if (x >= p.item_tiles || qb >= p.n_qb) {
       it.n_kv[x] = 0;
     } else if (p.causal) {
@@ -348,7 +357,8 @@ __device__ __forceinline__ void producer_role(SharedFwdT<kD>* sm, const FwdParam
           ok = false;
           continue;
         }
-        const int q_row = (it.b * p.Hq + it.hq) * p.S + (it.qb0 + x) * kBlockM;
+        const int q_row =
+            (it.b * p.Hq + it.hq + x * it.dhq) * p.S + (it.qb0 + x * it.dqb) * kBlockM;
         const uint32_t qf = smem_addr(&sm->q_full[x]);
         mbar_arrive_expect_tx(qf, kTile);
 #pragma unroll
@@ -394,12 +404,14 @@ __device__ __forceinline__ void producer_role(SharedFwdT<kD>* sm, const FwdParam
   }
 }
 
-// MMA issuer (a whole warp) for tiles x_lo..x_hi.  With two issuers the
-// K and V stages are released by both (count 2): the issuer of a tile that
-// does not read a block arrives at once.
-template <int kD, int kIssuers>
+// Single MMA issuer (a whole warp; one elected lane issues).  Per item and
+// key block j it waits for the step's V and K stages (and, at j = 0, the
+// tiles' Q), then issues for tile A and tile B the group PV_X(j-1), S_X(j),
+// each after its P (and, at j = 1, the epilogue's release of O).
+template <int kD>
 __device__ __forceinline__ void mma_role(SharedFwdT<kD>* sm, const FwdParams& p, uint32_t tmem,
-                                         int x_lo, int x_hi, volatile int* abort) {
+                                         volatile int* abort) {
+  constexpr int x_lo = 0, x_hi = 1;
   const uint64_t to = p.timeout_ns;
   int rc = 0;
   int pcnt[2] = {0, 0};  // P handoffs consumed
@@ -414,10 +426,7 @@ __device__ __forceinline__ void mma_role(SharedFwdT<kD>* sm, const FwdParams& p,
     for (int j = 0; ok && j <= n_b; ++j) {
       const int st_k = (rc + j) % kStagesK;
       const int st_v = (rc + j + kStagesV - 1) % kStagesV;
-      // The stages this step reads are awaited before anything is issued.
-      // An issuer also waits for a stage that only the other tile reads: it
-      // releases every stage, and its release must land in the stage's
-      // current phase, which it knows has begun once the stage is full.
+      // the stages this step reads are awaited before anything is issued
       const bool need_k = j < n_b;
       const bool need_v = j >= 1;
       if (need_v)
@@ -464,36 +473,18 @@ __device__ __forceinline__ void mma_role(SharedFwdT<kD>* sm, const FwdParams& p,
         }
       }
       if (!ok) break;
-      // ring releases: the K stage of block j once every S(j) of this issuer
-      // completed, the V stage of block j-1 once every PV(j-1) did
-      if (kIssuers == 1) {
-        if (j < n_b) tc_commit(smem_addr(&sm->k_empty[st_k]));
-        if (j >= 1) tc_commit(smem_addr(&sm->v_empty[st_v]));
-      } else {
-        const int n_x = x_lo ? it.n_kv[1] : it.n_kv[0];
-        if (j < n_b) {
-          if (j < n_x)
-            tc_commit(smem_addr(&sm->k_empty[st_k]));
-          else if (elect_one())
-            mbar_arrive(smem_addr(&sm->k_empty[st_k]));
-        }
-        if (j >= 1) {
-          if (j - 1 < n_x)
-            tc_commit(smem_addr(&sm->v_empty[st_v]));
-          else if (elect_one())
-            mbar_arrive(smem_addr(&sm->v_empty[st_v]));
-        }
-        __syncwarp();
-      }
+      // ring releases: the K stage of block j once every S(j) completed,
+      // the V stage of block j-1 once every PV(j-1) did
+      if (j < n_b) tc_commit(smem_addr(&sm->k_empty[st_k]));
+      if (j >= 1) tc_commit(smem_addr(&sm->v_empty[st_v]));
     }
     rc += n_b;
 #pragma unroll
     for (int x = 0; x < 2; ++x) qcnt[x] += it.n_kv[x] > 0 ? 1 : 0;
   }
   // every MMA issued must complete before TMEM is released
-  const int d = x_lo;
-  tc_commit(smem_addr(&sm->drain[d]));
-  drain_wait(smem_addr(&sm->drain[d]), 0, to, p.status);
+  tc_commit(smem_addr(&sm->drain[0]));
+  drain_wait(smem_addr(&sm->drain[0]), 0, to, p.status);
 }
 
 // Epilogue of one item (warps 8-11; thread r owns row r of both tiles):
@@ -521,9 +512,9 @@ __device__ __forceinline__ bool epilogue_item(SharedFwdT<kD>* sm, const FwdParam
     if (lane == 0) mbar_arrive(smem_addr(&sm->stats_free[x]));  // the softmax may write the next
     const float inv_l = 1.0f / l;
     // rows past S (a ragged last block) are computed but not stored
-    const int i_row = (it.qb0 + x) * kBlockM + r;
+    const int i_row = (it.qb0 + x * it.dqb) * kBlockM + r;
     const bool valid = i_row < p.S;
-    const int row = (it.b * p.Hq + it.hq) * p.S + i_row;
+    const int row = (it.b * p.Hq + it.hq + x * it.dhq) * p.S + i_row;
     uint4* orow = reinterpret_cast<uint4*>(p.o + static_cast<size_t>(row) * kD);
     float omax = 0.f;
 #pragma unroll
@@ -591,173 +582,166 @@ __device__ __forceinline__ void epilogue_role(SharedFwdT<kD>* sm, const FwdParam
   }
 }
 
-// Softmax of tile x (warps 4x..4x+3; thread = query row = TMEM lane).
+// The key blocks of one item for one tile's softmax warp (thread = query row
+// = TMEM lane).  kHilo: the exact pass (P = hi + lo).  Returns false if a
+// wait gave up; m_use and l hold the row's statistics on return.
+template <int kD, int kEmu, bool kHilo>
+__device__ __forceinline__ bool softmax_item(SharedFwdT<kD>* sm, const FwdParams& p, int x,
+                                             uint32_t s_t, uint32_t o_t, int n_x, int key_lim,
+                                             int j_mask, int lane, int& scnt, float& m_use,
+                                             float& l, volatile int* abort) {
+  const uint64_t to = p.timeout_ns;
+  const float sc = p.scale_log2;
+  m_use = -INFINITY;
+  l = 0.f;
+  for (int j = 0; j < n_x; ++j, ++scnt) {
+    bool ok = mbar_wait(smem_addr(&sm->s_full[x]), scnt & 1, abort, to, p.status, kSiteSoftmaxS);
+    if (!__all_sync(0xffffffffu, ok)) return false;
+    tc_fence_after();
+    // the row of S_X in 128 registers (fp32 bits)
+    uint32_t u[128];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) tmem_ld32(s_t + c * 32, &u[c * 32]);
+    tmem_wait_ld();
+#pragma unroll
+    for (int c = 0; c < 4; ++c) reg_dep32(&u[c * 32]);
+    // keys past the row's limit -> -inf (the causal diagonal, a ragged last
+    // key block)
+    if (j >= j_mask) {
+      const int lim = key_lim - j * kBlockN;
+#pragma unroll
+      for (int c = 0; c < 128; ++c)
+        if (c > lim) u[c] = 0xff800000u;  // -inf
+    }
+    // row max: 8 independent chains (chain t takes columns t, t + 8, ...) of
+    // 3-input max, then a tree
+    float mx8[8];
+#pragma unroll
+    for (int t = 0; t < 8; ++t)
+      mx8[t] = fmax3(__uint_as_float(u[t]), __uint_as_float(u[8 + t]), __uint_as_float(u[16 + t]));
+#pragma unroll
+    for (int c = 24; c < 120; c += 16)
+#pragma unroll
+      for (int t = 0; t < 8; ++t)
+        mx8[t] = fmax3(mx8[t], __uint_as_float(u[c + t]), __uint_as_float(u[c + 8 + t]));
+#pragma unroll
+    for (int t = 0; t < 8; ++t) mx8[t] = fmaxf(mx8[t], __uint_as_float(u[120 + t]));
+    const float cand = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
+                             fmaxf(mx8[6], mx8[7])) * sc;
+    if (j == 0) {
+      m_use = cand;
+    } else {
+      const bool grow = cand > m_use + kRescaleLog2;
+      if (__any_sync(0xffffffffu, grow)) {
+        // O_X holds P(j-1) V_{j-1} already (it completed before S(j))
+        const float alpha = grow ? ex2_approx(m_use - cand) : 1.0f;
+#pragma unroll 1
+        for (int c = 0; c < kD / 32; ++c) {
+          uint32_t wv[32];
+          tmem_ld32(o_t + c * 32, wv);
+          tmem_wait_ld();
+          reg_dep32(wv);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) wv[i] = __float_as_uint(__uint_as_float(wv[i]) * alpha);
+          tmem_st32(o_t + c * 32, wv);
+        }
+        if (grow) {
+          l *= alpha;
+          m_use = cand;
+        }
+      }
+    }
+    const float neg_m = -m_use;
+    float lp[4] = {0.f, 0.f, 0.f, 0.f};
+    if constexpr (!kHilo) {
+      // P rounded to fp16; l sums exactly the rounded values.  In every 16
+      // columns, kEmu pairs take 2^x from the FMA-pipe polynomial and the rest
+      // from the MUFU unit.
+      const float2 sc2 = make_float2(sc, sc);
+      const float2 nm2 = make_float2(neg_m, neg_m);
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        uint32_t ph[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float2 s2 = make_float2(__uint_as_float(u[c * 16 + 2 * i]),
+                                        __uint_as_float(u[c * 16 + 2 * i + 1]));
+          const float2 x2 = __ffma2_rn(s2, sc2, nm2);
+          float2 p2;
+          if (i < kEmu) {
+            p2 = exp2_poly2(x2);
+          } else {
+            p2.x = ex2_approx(x2.x);
+            p2.y = ex2_approx(x2.y);
+          }
+          ph[i] = pack_half2(p2.x, p2.y);
+          lp[i & 3] = add_half2_f32(ph[i], lp[i & 3]);
+        }
+        tmem_st8(s_t + c * 8, ph);
+      }
+    } else {
+      // P = hi + lo, both fp16: hi over columns [0,64), lo over [64,128); l
+      // sums the fp32 p the two parts represent
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        uint32_t ph[8], pl[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float p0 = ex2_approx(fmaf(__uint_as_float(u[c * 16 + 2 * i]), sc, neg_m));
+          const float p1 = ex2_approx(fmaf(__uint_as_float(u[c * 16 + 2 * i + 1]), sc, neg_m));
+          ph[i] = pack_half2(p0, p1);
+          const float2 h = __half22float2(*reinterpret_cast<const __half2*>(&ph[i]));
+          pl[i] = pack_half2(p0 - h.x, p1 - h.y);
+          lp[i & 3] += p0 + p1;
+        }
+        tmem_st8(s_t + c * 8, ph);
+        tmem_st8(s_t + 64 + c * 8, pl);
+      }
+    }
+    l += (lp[0] + lp[1]) + (lp[2] + lp[3]);
+    tmem_wait_st();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(smem_addr(&sm->p_full[x]));
+  }
+  return true;
+}
+
+// Softmax of tile x (warps 4x..4x+3).
 template <int kD, int kEmu>
 __device__ __forceinline__ void softmax_role(SharedFwdT<kD>* sm, const FwdParams& p, uint32_t tmem,
                                              int warp, int lane, volatile int* abort) {
-  const uint64_t to = p.timeout_ns;
   const int x = warp >> 2;  // tile
   const int r = (warp & 3) * 32 + lane;
   const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
   const uint32_t s_t = lane_base + tmem_s_col(x);
   const uint32_t o_t = lane_base + tmem_o_col(x);
-  const float sc = p.scale_log2;
   int scnt = 0;
   int acnt = 0;  // items so far in which this tile was active
   bool ok = true;
   ItemWalk w;
   int item;
   while (ok && (item = walk_next(w, p, sm, abort, ok, kSiteSoftmaxRedo)) >= 0) {
-    const bool hilo = w.exact;
     const Item it = decode_item(p, item);
     const int n_x = x ? it.n_kv[1] : it.n_kv[0];
     if (n_x == 0) continue;
     // the last key this row sees: row + off (causal), and never past Sk (a
     // ragged last key block reads the next head's rows, or zero fill past
     // the tensor); rows past S are computed but not stored
-    const int i_row = (it.qb0 + x) * kBlockM + r;
+    const int i_row = (it.qb0 + x * it.dqb) * kBlockM + r;
     const int key_lim = p.causal ? min(i_row + p.off, p.Sk - 1) : p.Sk - 1;
     // key_lim grows with the lane, so from this block on (warp-uniform) some
     // lane of the warp has keys to mask
     const int j_mask = (__shfl_sync(0xffffffffu, key_lim, 0) + 1) / kBlockN;
-    float m_use = -INFINITY;
-    float l = 0.f;
-    for (int j = 0; j < n_x; ++j, ++scnt) {
-      ok = mbar_wait(smem_addr(&sm->s_full[x]), scnt & 1, abort, to, p.status, kSiteSoftmaxS);
-      if (!__all_sync(0xffffffffu, ok)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      // the row of S_X in 128 registers (fp32 bits), loaded in two halves
-      // so the max of the first half overlaps the load of the second
-      uint32_t u[128];
-      tmem_ld32(s_t, &u[0]);
-      tmem_ld32(s_t + 32, &u[32]);
-      tmem_wait_ld();
-      reg_dep32(&u[0]);
-      reg_dep32(&u[32]);
-      tmem_ld32(s_t + 64, &u[64]);
-      tmem_ld32(s_t + 96, &u[96]);
-      // keys past the row's limit -> -inf (the causal diagonal, a ragged
-      // last key block)
-      const bool masked = j >= j_mask;
-      const int lim = key_lim - j * kBlockN;
-      if (masked) {
-#pragma unroll
-        for (int c = 0; c < 64; ++c)
-          if (c > lim) u[c] = 0xff800000u;  // -inf
-      }
-      // row max: 8 independent chains (chain t takes columns t, t + 8, ...)
-      // of 3-input max, then a tree
-      float mx8[8];
-#pragma unroll
-      for (int t = 0; t < 8; ++t)
-        mx8[t] = fmax3(__uint_as_float(u[t]), __uint_as_float(u[8 + t]),
-                       __uint_as_float(u[16 + t]));
-#pragma unroll
-      for (int c = 24; c < 56; c += 16)
-#pragma unroll
-        for (int t = 0; t < 8; ++t)
-          mx8[t] = fmax3(mx8[t], __uint_as_float(u[c + t]), __uint_as_float(u[c + 8 + t]));
-#pragma unroll
-      for (int t = 0; t < 8; ++t) mx8[t] = fmaxf(mx8[t], __uint_as_float(u[56 + t]));
-      tmem_wait_ld();
-      reg_dep32(&u[64]);
-      reg_dep32(&u[96]);
-      if (masked) {
-#pragma unroll
-        for (int c = 64; c < 128; ++c)
-          if (c > lim) u[c] = 0xff800000u;
-      }
-#pragma unroll
-      for (int c = 64; c < 128; c += 16)
-#pragma unroll
-        for (int t = 0; t < 8; ++t)
-          mx8[t] = fmax3(mx8[t], __uint_as_float(u[c + t]), __uint_as_float(u[c + 8 + t]));
-      const float cand = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
-                               fmaxf(mx8[6], mx8[7])) * sc;
-      if (j == 0) {
-        m_use = cand;
-      } else {
-        const bool grow = cand > m_use + kRescaleLog2;
-        if (__any_sync(0xffffffffu, grow)) {
-          // O_X holds P(j-1) V_{j-1} already (it completed before S(j))
-          const float alpha = grow ? ex2_approx(m_use - cand) : 1.0f;
-#pragma unroll 1
-          for (int c = 0; c < kD / 32; ++c) {
-            uint32_t wv[32];
-            tmem_ld32(o_t + c * 32, wv);
-            tmem_wait_ld();
-            reg_dep32(wv);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) wv[i] = __float_as_uint(__uint_as_float(wv[i]) * alpha);
-            tmem_st32(o_t + c * 32, wv);
-          }
-          if (grow) {
-            l *= alpha;
-            m_use = cand;
-          }
-        }
-      }
-      const float neg_m = -m_use;
-      float lp[4] = {0.f, 0.f, 0.f, 0.f};
-      if (!hilo) {
-        // P rounded to fp16; l sums exactly the rounded values.  In every 16
-        // columns, kEmu pairs take 2^x from the FMA-pipe polynomial and the
-        // rest from the MUFU unit.
-        const float2 sc2 = make_float2(sc, sc);
-        const float2 nm2 = make_float2(neg_m, neg_m);
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          uint32_t ph[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const float2 s2 = make_float2(__uint_as_float(u[c * 16 + 2 * i]),
-                                          __uint_as_float(u[c * 16 + 2 * i + 1]));
-            const float2 x2 = __ffma2_rn(s2, sc2, nm2);
-            float2 p2;
-            if (i < kEmu) {
-              p2 = exp2_poly2(x2);
-            } else {
-              p2.x = ex2_approx(x2.x);
-              p2.y = ex2_approx(x2.y);
-            }
-            ph[i] = pack_half2(p2.x, p2.y);
-            lp[i & 3] = add_half2_f32(ph[i], lp[i & 3]);
-          }
-          tmem_st8(s_t + c * 8, ph);
-        }
-      } else {
-        // P = hi + lo, both fp16: hi over columns [0,64), lo over [64,128);
-        // l sums the fp32 p the two parts represent
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          uint32_t ph[8], pl[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const float p0 = ex2_approx(fmaf(__uint_as_float(u[c * 16 + 2 * i]), sc, neg_m));
-            const float p1 = ex2_approx(fmaf(__uint_as_float(u[c * 16 + 2 * i + 1]), sc, neg_m));
-            ph[i] = pack_half2(p0, p1);
-            const float2 h = __half22float2(*reinterpret_cast<const __half2*>(&ph[i]));
-            pl[i] = pack_half2(p0 - h.x, p1 - h.y);
-            lp[i & 3] += p0 + p1;
-          }
-          tmem_st8(s_t + c * 8, ph);
-          tmem_st8(s_t + 64 + c * 8, pl);
-        }
-      }
-      l += (lp[0] + lp[1]) + (lp[2] + lp[3]);
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_addr(&sm->p_full[x]));
-    }
+    float m_use, l;
+    ok = w.exact ? softmax_item<kD, kEmu, true>(sm, p, x, s_t, o_t, n_x, key_lim, j_mask, lane,
+                                                 scnt, m_use, l, abort)
+                 : softmax_item<kD, kEmu, false>(sm, p, x, s_t, o_t, n_x, key_lim, j_mask, lane,
+                                                  scnt, m_use, l, abort);
     if (!ok) break;
     // the epilogue must have read this tile's previous statistics
-    ok = acnt == 0 ||
-         mbar_wait(smem_addr(&sm->stats_free[x]), (acnt - 1) & 1, abort, to, p.status,
-                   kSiteSoftmaxStats);
+    ok = acnt == 0 || mbar_wait(smem_addr(&sm->stats_free[x]), (acnt - 1) & 1, abort,
+                                p.timeout_ns, p.status, kSiteSoftmaxStats);
     if (!__all_sync(0xffffffffu, ok)) {
       ok = false;
       break;
@@ -771,14 +755,12 @@ __device__ __forceinline__ void softmax_role(SharedFwdT<kD>* sm, const FwdParams
 }
 
 // kD: the head dimension, 64 or 128.  kEmu: FMA-pipe exponentials per 8
-// column pairs in the fast pass.  kIssuers: MMA-issuing warps, 1 (both tiles)
-// or 2 (one per tile).
-template <int kD = 128, int kEmu = 0, int kIssuers = 1>
+// column pairs in the fast pass.
+template <int kD = 128, int kEmu = 0>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
   static_assert(kEmu >= 0 && kEmu <= kEmuMax, "kEmu: 0..4");
-  static_assert(kIssuers == 1 || kIssuers == 2, "one or two MMA issuers");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   SharedFwdT<kD>* sm = reinterpret_cast<SharedFwdT<kD>*>(smem_raw);
   const int warp = threadIdx.x >> 5;
@@ -805,11 +787,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int s = 0; s < kStagesK; ++s) {
       mbar_init(smem_addr(&sm->k_full[s]), 1);
-      mbar_init(smem_addr(&sm->k_empty[s]), kIssuers);
+      mbar_init(smem_addr(&sm->k_empty[s]), 1);
     }
     for (int s = 0; s < kStagesV; ++s) {
       mbar_init(smem_addr(&sm->v_full[s]), 1);
-      mbar_init(smem_addr(&sm->v_empty[s]), kIssuers);
+      mbar_init(smem_addr(&sm->v_empty[s]), 1);
     }
     mbar_init(smem_addr(&sm->redo_ready), 4);
     for (int i = 0; i < kRedoWords; ++i) sm->redo_bits[i] = 0;
@@ -837,9 +819,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) producer_role<kD>(sm, p, &tm_q, warp == kProducerVWarp ? &tm_v : &tm_k,
                                        warp == kProducerVWarp, abort);
     } else if (warp == kMmaWarp) {
-      mma_role<kD, kIssuers>(sm, p, tmem, 0, kIssuers == 1 ? 1 : 0, abort);
-    } else if (kIssuers == 2) {  // warp 15
-      mma_role<kD, kIssuers>(sm, p, tmem, 1, 1, abort);
+      mma_role<kD>(sm, p, tmem, abort);
     }
     __syncwarp();
   } else if (warp >= kEpilogueWarp0) {

@@ -108,14 +108,24 @@ attn_status attn_fwd_qk(const void* q, const void* k, const void* v, void* o, fl
  * is that the best tiling / pipeline choice of an attention kernel is found by
  * profiling candidates on the target GPU (PipeThreader pages, sections 核心方法
  * and 设计取舍: a joint tile + pipeline search whose greedy choices are checked
- * by profiling); this library keeps that idea as a small build-time table.  The fused kernel
- * is compiled in attn_variant_count() variants along two axes of its
- * pipeline: how many warps issue the tensor-core MMAs (one for both 128-row
- * tiles of a work item, or one per tile) and how many of every 16
+ * by profiling); this library keeps that idea as a small build-time table.
+ * The fused pass is compiled in attn_variant_count() variants, the product of
+ * two axes.  The pipeline structure (variant v, structure v / 5):
+ *   0 "pingpong,row_pairs"   two 128-row tiles of one query head (256 rows)
+ *                            take turns on the tensor core, 128-key blocks;
+ *   1 "pingpong,head_pairs"  the same schedule with the two tiles on the same
+ *                            128 rows of two query heads of one group (falls
+ *                            back to row pairs when Hq/Hkv is odd);
+ *   2 "dbuf,softmax_split=1" one 128-row tile, S double-buffered in TMEM so
+ *                            the softmax of one key block overlaps the MMAs
+ *                            of the next (64-key blocks at D = 256);
+ *   3 "dbuf,softmax_split=2" as 2, with two softmax warps per row, each on
+ *                            half of a key block.
+ * At D = 256 every structure runs as structure 2.  The second
+ * axis, N = v % 5 ("fma_exp2_pairs=N/8"), is how many of every 16
  * exponentials of the softmax an FMA-pipe polynomial evaluates instead of the
- * MUFU unit (variant v: name "mma_issuers=I,fma_exp2_pairs=N/8" with
- * I = 1 + v / 5, N = v % 5; the issuers axis changes no result, and the
- * polynomial's relative error 8e-5 is well inside fp16 rounding of P).  The
+ * MUFU unit (relative error 8e-5, well inside the fp16 rounding of P).  The
+ * structures change the work order, not the arithmetic of a row.  The
  * package's tuner
  * (python -m dnn_compiler_pipelining_b200.tune) times every variant per
  * shape class on a B200 and writes the table compiled into the library;

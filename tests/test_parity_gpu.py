@@ -458,13 +458,14 @@ def test_fma_pipe_exp2_error_bound():
     assert torch.all(lo >= 0) and torch.all(lo < 2.0 ** -124), lo
 
 
-# Every fused-kernel variant (two-tile ping-pong with one or two MMA-issuing
-# warps, one tile with S double-buffered and one or two softmax warps per lane
+# Every fused-kernel variant (two-tile ping-pong over row pairs or head
+# pairs, one tile with S double-buffered and one or two softmax warps per lane
 # quadrant, x 0..4 of every 8 exponential pairs from the FMA-pipe polynomial)
 # through attn_fwd_variant, against the oracle: both head dims, a ragged
 # tail, logits of standard deviation 1 and 16, one-tile and two-tile items.
 VARIANT_CASES = [(2, 4, 2, 383, 128, 1.0), (1, 8, 2, 512, 128, 4.0), (2, 4, 2, 329, 64, 1.0),
-                 (1, 4, 2, 640, 64, 4.0), (1, 64, 8, 700, 128, 1.0)]
+                 (1, 4, 2, 640, 64, 4.0), (1, 64, 8, 700, 128, 1.0), (2, 48, 8, 520, 128, 4.0),
+                 (1, 96, 8, 384, 64, 1.0)]
 
 
 def _variant_check(q, k, v, causal, variant, what):

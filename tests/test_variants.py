@@ -42,7 +42,7 @@ def test_count_and_names(lib):
     n = attn.variant_count()
     assert n == 20
     names = [attn.variant_name(i) for i in range(n)]
-    structures = ["pingpong,mma_issuers=1", "pingpong,mma_issuers=2", "dbuf,softmax_split=1",
+    structures = ["pingpong,row_pairs", "pingpong,head_pairs", "dbuf,softmax_split=1",
                   "dbuf,softmax_split=2"]
     assert names == ["%s,fma_exp2_pairs=%d/8" % (structures[i // 5], i % 5) for i in range(20)]
     assert attn.variant_name(-1) is None and attn.variant_name(n) is None
@@ -151,7 +151,7 @@ def test_tuner_writes_a_table_the_library_format_accepts(tmp_path, monkeypatch):
     tune.main(["--table", str(table), "--report", str(report)])
     text = open(table).read()
     rules = table_rules(str(table))
-    assert len(fake) == 20
+    assert len(fake) == 30   # D in {64, 128, 256} x causal x 5 sequence lengths
     assert expected_variant(rules, 64, 1, 8192) == 2 and expected_variant(rules, 64, 1, 2048) == 2
     # 1448 is the geometric midpoint of 1024 and 2048: the 2048 rule starts just above it
     assert expected_variant(rules, 64, 1, 1448) == 0 and expected_variant(rules, 64, 1, 1449) == 2
