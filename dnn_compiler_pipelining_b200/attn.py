@@ -75,6 +75,8 @@ def load() -> ctypes.CDLL:
     lib.attn_set_wait_timeout_ns.restype = u64
     lib.attn_selftest_exp2.argtypes = [vp, vp, i, vp]
     lib.attn_selftest_exp2.restype = i
+    lib.attn_selftest_fastdiv.argtypes = [ctypes.c_uint32, vp, vp, i, i, vp]
+    lib.attn_selftest_fastdiv.restype = i
     lib.attn_selftest_wait_timeout.argtypes = [u64, vp]
     lib.attn_selftest_wait_timeout.restype = i
     lib.attn_status_string.argtypes = [i]
@@ -297,6 +299,23 @@ def set_wait_timeout_ns(ns: int) -> int:
 
 def selftest_wait_timeout(ns: int, stream=None) -> int:
     return int(load().attn_selftest_wait_timeout(int(ns), _stream_ptr(stream)))
+
+
+def selftest_fastdiv(d: int, n: torch.Tensor) -> torch.Tensor:
+    """n // d through the kernels' multiply-shift division; n is an int32
+    tensor of values in [0, 2^31), on the CPU (host arithmetic) or on the GPU
+    (device arithmetic)."""
+    n = n.contiguous()
+    if n.dtype != torch.int32:
+        raise ValueError("n must be int32")
+    q = torch.empty_like(n)
+    st = load().attn_selftest_fastdiv(int(d), n.data_ptr(), q.data_ptr(), n.numel(),
+                                      1 if n.is_cuda else 0, _stream_ptr(None) if n.is_cuda else None)
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_selftest_fastdiv")
+    if n.is_cuda:
+        torch.cuda.current_stream().synchronize()
+    return q
 
 
 def selftest_exp2(x: torch.Tensor) -> torch.Tensor:

@@ -276,6 +276,11 @@ FwdParams make_params(void* o, float* lse, unsigned int* status, int B, int Hq, 
   // once, so it is used only when all of K and V stay resident in L2.
   const double kv_bytes = 2.0 * B * Hkv * static_cast<double>(Sk) * D * 2;
   p.order = (causal && kv_bytes <= 0.5 * l2) ? 1 : 0;
+  const int members = p.pair_heads ? p.group / 2 : p.group;
+  p.div_members = make_fastdiv(static_cast<uint32_t>(members));
+  p.div_major = make_fastdiv(static_cast<uint32_t>(
+      p.order == 0 ? members * p.n_qi : static_cast<long long>(B) * Hkv * members));
+  p.div_hkv = make_fastdiv(static_cast<uint32_t>(Hkv));
   p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
   p.timeout_ns = g_timeout_ns.load();
   return p;
@@ -627,6 +632,31 @@ extern "C" attn_status attn_selftest_exp2(const float* x, float* y, int n, void*
   if (st != ATTN_OK) return st;
   const int pairs = (n + 1) / 2;
   selftest_exp2_kernel<<<(pairs + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+namespace attn_b200 {
+__global__ void selftest_fastdiv_kernel(FastDiv f, const uint32_t* n, uint32_t* q, int count) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < count) q[i] = fast_div(n[i], f);
+}
+}  // namespace attn_b200
+
+extern "C" attn_status attn_selftest_fastdiv(uint32_t d, const uint32_t* n, uint32_t* q,
+                                             int count, int on_device, void* stream) {
+  if (d == 0 || count < 0) return ATTN_ERR_SHAPE;
+  if (count == 0) return ATTN_OK;
+  if (!n || !q) return ATTN_ERR_NULL;
+  const FastDiv f = make_fastdiv(d);
+  if (!on_device) {
+    for (int i = 0; i < count; ++i) q[i] = fast_div(n[i], f);
+    return ATTN_OK;
+  }
+  int dev = 0;
+  attn_status st = device_setup(&dev);
+  if (st != ATTN_OK) return st;
+  selftest_fastdiv_kernel<<<(count + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      f, n, q, count);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 

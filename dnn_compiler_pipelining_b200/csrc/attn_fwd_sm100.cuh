@@ -93,6 +93,35 @@ __device__ __forceinline__ uint32_t tmem_o_col(int x) { return 256u + x * 128u; 
 // instead of the MUFU unit (the kernel's kEmu argument).
 constexpr int kEmuMax = 4;
 
+// Division by a divisor fixed for the launch, without the hardware integer
+// divide: that goes through the reciprocal of the MUFU unit, which the
+// softmax keeps busy with exponentials, and measured ~1800 cycles for the
+// three divisions of an item decode.  q = (umulhi(n, m) + n) >> s, exact for
+// 0 <= n < 2^31, with s = ceil(log2 d) and m = floor(2^32 (2^s - d) / d) + 1:
+// the round-up multiplier of Granlund and Montgomery ("Division by invariant
+// integers using multiplication", PLDI 1994), 2^32 + m = floor(2^(32+s)/d)+1,
+// split so that the product fits 32-bit operations (n < 2^31 keeps the sum
+// below 2^32).
+struct FastDiv {
+  uint32_t d, m, s;
+};
+
+inline FastDiv make_fastdiv(uint32_t d) {
+  uint32_t s = 0;
+  while ((1ull << s) < d) ++s;
+  const uint64_t m = ((1ull << 32) * ((1ull << s) - d)) / d + 1;
+  return {d, static_cast<uint32_t>(m), s};
+}
+
+__host__ __device__ __forceinline__ uint32_t fast_div(uint32_t n, const FastDiv& f) {
+#ifdef __CUDA_ARCH__
+  const uint32_t hi = __umulhi(n, f.m);
+#else
+  const uint32_t hi = static_cast<uint32_t>((static_cast<uint64_t>(n) * f.m) >> 32);
+#endif
+  return (hi + n) >> f.s;
+}
+
 struct FwdParams {
   __half* o;
   float* lse;
@@ -110,6 +139,9 @@ struct FwdParams {
   int n_qi;              // items per (batch, head or head pair)
   int n_items;
   int order;             // 0: kv-head major, round robin; 1: longest first, snake
+  FastDiv div_major;     // items per kv head (order 0) or per row block (order 1)
+  FastDiv div_members;   // query heads (or head pairs) per kv group
+  FastDiv div_hkv;       // Hkv
   float scale_log2;      // log2(e) / sqrt(D)
   unsigned long long timeout_ns;
 };
@@ -175,27 +207,27 @@ struct Item {
 
 __device__ __forceinline__ Item decode_item(const FwdParams& p, int id) {
   // the query heads (or head pairs) of a kv group an item can start at
-  const int members = p.pair_heads ? p.group / 2 : p.group;
+  const int members = static_cast<int>(p.div_members.d);
+  const int major = static_cast<int>(p.div_major.d);
   int qi, kvh, member;
   if (p.order == 0) {
     // kv-head major; inside a kv head: row blocks from last to first, the
     // group's query heads adjacent
-    const int per_kv = members * p.n_qi;
-    kvh = id / per_kv;
-    const int rem = id - kvh * per_kv;
-    qi = p.n_qi - 1 - rem / members;
-    member = rem - (rem / members) * members;
+    kvh = static_cast<int>(fast_div(id, p.div_major));
+    const int rem = id - kvh * major;
+    const int t = static_cast<int>(fast_div(rem, p.div_members));
+    qi = p.n_qi - 1 - t;
+    member = rem - t * members;
   } else {
     // row blocks from last (longest) to first; inside one, kv-head major
-    const int heads = p.B * p.Hkv * members;
-    const int r = id / heads;
-    const int rem = id - r * heads;
+    const int r = static_cast<int>(fast_div(id, p.div_major));
+    const int rem = id - r * major;
     qi = p.n_qi - 1 - r;
-    kvh = rem / members;
+    kvh = static_cast<int>(fast_div(rem, p.div_members));
     member = rem - kvh * members;
   }
   Item it;
-  it.b = kvh / p.Hkv;
+  it.b = static_cast<int>(fast_div(kvh, p.div_hkv));
   it.g = kvh - it.b * p.Hkv;
   it.dhq = p.pair_heads;
   it.dqb = p.pair_heads ? 0 : 1;

@@ -258,6 +258,19 @@ attn_status attn_noalloc_status(void* stream, uint32_t* site, uint64_t* exact_it
  */
 attn_status attn_selftest_exp2(const float* x, float* y, int n, void* stream);
 
+/*
+ * attn_selftest_fastdiv -- the division by a launch-time constant that the
+ * kernels use to decode their work items (a multiply-high and a shift in
+ * place of the hardware divide; Granlund and Montgomery, "Division by
+ * invariant integers using multiplication", PLDI 1994): q[i] = n[i] / d for
+ * count values 0 <= n[i] < 2^31, d >= 1.  on_device = 0: n and q are host
+ * arrays and the host evaluates the same arithmetic, synchronously;
+ * on_device = 1: device arrays, evaluated by a kernel on `stream`
+ * (asynchronous).  ATTN_ERR_SHAPE for d == 0 or count < 0.
+ */
+attn_status attn_selftest_fastdiv(uint32_t d, const uint32_t* n, uint32_t* q, int count,
+                                  int on_device, void* stream);
+
 /* Human-readable name of a status code (static storage, never NULL). */
 const char* attn_status_string(attn_status status);
 

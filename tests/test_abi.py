@@ -5,6 +5,7 @@ import ctypes
 import os
 import re
 
+import numpy as np
 import pytest
 import torch
 
@@ -109,3 +110,34 @@ def test_timeout_setting_roundtrip(lib):
     prev = attn.set_wait_timeout_ns(5_000_000)
     assert attn.set_wait_timeout_ns(10) == 5_000_000   # clamped up to 1 ms on the next set
     assert attn.set_wait_timeout_ns(prev) == 1_000_000
+
+
+def _fastdiv_cases():
+    """Divisors 1..300, powers of two and their neighbours, and large odd
+    values; numerators at 0, 1, multiples of d and their neighbours, the top
+    of the range (2^31 - 1) and seeded random values."""
+    rng = np.random.default_rng(5)
+    ds = list(range(1, 301)) + [2 ** k + e for k in range(9, 31) for e in (-1, 0, 1)]
+    ds += [int(x) for x in rng.integers(1, 2 ** 31 - 1, 40)]
+    for d in ds:
+        ns = [0, 1, 2 ** 31 - 1, 2 ** 31 - 2, d - 1, d, d + 1]
+        ks = np.unique(np.concatenate([np.arange(0, 50), rng.integers(0, (2 ** 31 - 1) // d + 1, 50)]))
+        for k in ks:
+            for e in (-1, 0, 1):
+                ns.append(int(k) * d + e)
+        ns += [int(x) for x in rng.integers(0, 2 ** 31, 200)]
+        ns = np.array([x for x in ns if 0 <= x < 2 ** 31], dtype=np.int64)
+        yield d, ns
+
+
+def test_fastdiv_host_matches_floor_division(lib):
+    """The multiply-shift division the kernels use to decode work items is
+    exact floor division for every numerator below 2^31 (host evaluation of
+    the same formula)."""
+    for d, ns in _fastdiv_cases():
+        q = attn.selftest_fastdiv(d, torch.from_numpy(ns.astype(np.int32)))
+        assert np.array_equal(q.numpy().astype(np.int64), ns // d), d
+    n = torch.zeros(4, dtype=torch.int32)
+    assert lib.attn_selftest_fastdiv(0, n.data_ptr(), n.data_ptr(), 4, 0, None) == 2  # d == 0
+    assert lib.attn_selftest_fastdiv(3, None, None, 4, 0, None) == 1
+    assert lib.attn_selftest_fastdiv(3, None, None, 0, 0, None) == 0

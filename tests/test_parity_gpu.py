@@ -439,6 +439,21 @@ def test_call_split_into_launches():
     torch.cuda.empty_cache()
 
 
+def test_fastdiv_device_matches_floor_division():
+    """The kernels' item decode divides with a multiply-high and a shift; on
+    the device it is exact floor division for numerators below 2^31."""
+    rng = np.random.default_rng(11)
+    ds = list(range(1, 130)) + [255, 256, 257, 4095, 4096, 4097, 2 ** 30 + 1, 2 ** 31 - 1]
+    ds += [int(x) for x in rng.integers(1, 2 ** 31 - 1, 16)]
+    for d in ds:
+        ns = np.concatenate([np.arange(0, 4096), rng.integers(0, 2 ** 31, 8192),
+                             np.array([2 ** 31 - 1, 2 ** 31 - 2]),
+                             (np.arange(1, 64) * d - 1) % 2 ** 31, (np.arange(1, 64) * d) % 2 ** 31])
+        n = torch.from_numpy(ns.astype(np.int32)).cuda()
+        q = attn.selftest_fastdiv(d, n).cpu().numpy().astype(np.int64)
+        assert np.array_equal(q, ns.astype(np.int64) // d), d
+
+
 def test_fma_pipe_exp2_error_bound():
     """The polynomial 2^x available to the fused pass for part of its
     exponentials: relative error <= 8e-5 against fp64 exp2 for x in
