@@ -52,11 +52,11 @@ def test_table_well_formed(lib):
     rules = table_rules()
     n = attn.variant_count()
     for d, c, lo, hi, var in rules:
-        assert d in (64, 128) and c in (0, 1)
+        assert d in (64, 128, 256) and c in (0, 1)
         assert 1 <= lo <= hi <= 2 ** 31 - 1
         assert 0 <= var < n
     # within one (D, causal) class the S ranges do not overlap
-    for D in (64, 128):
+    for D in (64, 128, 256):
         for c in (0, 1):
             spans = sorted((lo, hi) for d, cc, lo, hi, _ in rules if d == D and cc == c)
             for (lo0, hi0), (lo1, hi1) in zip(spans, spans[1:]):
@@ -69,7 +69,7 @@ def test_select_follows_table(lib):
               2896, 2897, 4096, 5792, 5793, 8192, 16384, 65536}
     for lo_hi in rules:
         probes |= {lo_hi[2], lo_hi[3], max(1, lo_hi[2] - 1), lo_hi[3] + 1}
-    for D in (64, 128):
+    for D in (64, 128, 256):
         for causal in (0, 1):
             for Sk in sorted(probes):
                 if Sk < 1 or Sk > 2 ** 20:
