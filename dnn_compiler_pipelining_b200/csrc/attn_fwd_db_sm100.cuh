@@ -482,7 +482,9 @@ __device__ __forceinline__ bool epilogue_item(SharedDb<kD, kSplit>* sm, const Fw
   const int i_row = it.qb0 * kBlockM + r;
   const bool valid = i_row < p.S;
   const int row = (it.b * p.Hq + it.hq) * p.S + i_row;
-  uint4* orow = reinterpret_cast<uint4*>(p.o + static_cast<size_t>(row) * kD);
+  __half* orow = p.o + static_cast<size_t>(row) * kD;
+  // full-sector stores when O is 32-byte aligned (rows are kD * 2 bytes apart)
+  const bool sector_aligned = (reinterpret_cast<uintptr_t>(p.o) & 31u) == 0;
   float omax = 0.f;
 #pragma unroll 4
   for (int c = 0; c < kD / 16; ++c) {
@@ -490,20 +492,22 @@ __device__ __forceinline__ bool epilogue_item(SharedDb<kD, kSplit>* sm, const Fw
     tmem_ld16(lane_base + C::kTmemO + c * 16, wv);
     tmem_wait_ld();
     reg_dep16(wv);
+    uint32_t pk[8];
 #pragma unroll
-    for (int v4 = 0; v4 < 2; ++v4) {
-      float f[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        f[e] = __uint_as_float(wv[v4 * 8 + e]) * inv_l;
-        omax = fmaxf(omax, fabsf(f[e]));
+    for (int e = 0; e < 8; ++e) {
+      const float f0 = __uint_as_float(wv[2 * e]) * inv_l;
+      const float f1 = __uint_as_float(wv[2 * e + 1]) * inv_l;
+      omax = fmax3(omax, fabsf(f0), fabsf(f1));
+      pk[e] = pack_half2(f0, f1);
+    }
+    if (valid) {
+      if (sector_aligned) {
+        st_global_v8(orow + c * 16, pk);
+      } else {
+        uint4* o16 = reinterpret_cast<uint4*>(orow + c * 16);
+        o16[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        o16[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
       }
-      uint4 pk;
-      pk.x = pack_half2(f[0], f[1]);
-      pk.y = pack_half2(f[2], f[3]);
-      pk.z = pack_half2(f[4], f[5]);
-      pk.w = pack_half2(f[6], f[7]);
-      if (valid) orow[c * 2 + v4] = pk;
     }
   }
   tc_fence_before();

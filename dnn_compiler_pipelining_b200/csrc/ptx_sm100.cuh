@@ -248,6 +248,14 @@ __device__ __forceinline__ void tc_commit(uint32_t bar) {
       : "memory");
 }
 
+// One 32-byte (full sector) store of eight 32-bit words; `p` must be 32-byte
+// aligned.
+__device__ __forceinline__ void st_global_v8(void* p, const uint32_t (&r)[8]) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(r[0]),
+               "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
+}
+
 // ===========================================================================
 // tcgen05: TMEM <-> registers (32x32b shapes: thread t of the warp holds
 // lane (base lane + t), consecutive 32-bit columns)

@@ -248,6 +248,23 @@ def test_deterministic():
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
 
 
+@pytest.mark.parametrize("D", [64, 128, 256])
+def test_output_only_16_byte_aligned(D):
+    """O at an address that is 16- but not 32-byte aligned goes out as 16-byte
+    stores instead of full-sector ones; it must hold exactly what the call
+    with an aligned O stores, and nothing past it may change."""
+    B, Hq, Hkv, S = 2, 8, 2, 300
+    q, k, v = make_qkv(B, Hq, Hkv, S, D, seed=5, device="cuda")
+    o1, l1 = attn.attn_fwd(q, k, v, True)
+    buf = torch.full((q.numel() + 16,), 7.0, dtype=torch.float16, device="cuda")
+    o2 = buf[8:8 + q.numel()].view_as(q)  # +16 bytes from a 256-byte aligned base
+    assert o2.data_ptr() % 32 == 16
+    _, l2 = attn.attn_fwd(q, k, v, True, o=o2)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+    assert torch.all(buf[:8] == 7.0) and torch.all(buf[8 + q.numel():] == 7.0)
+
+
 def test_concurrent_streams():
     """Calls on two streams run at the same time, each with its own status
     block: large-V inputs (every item recomputed by the exact pass) on one
