@@ -49,11 +49,28 @@ def attn_flops(B, Hq, S, D, causal):
     return f / 2 if causal else f
 
 
+def n_items(w, sms=148):
+    """Work items of one attn_fwd call of this workload, for the variant the
+    library's table picks: 256-row items (two 128-row tiles of one head, or
+    the same rows of two heads), or 128-row items for the double-buffered
+    kernel and for calls whose 256-row items would leave SMs idle."""
+    from dnn_compiler_pipelining_b200 import attn
+    B, Hq, Hkv, S, D = w["B"], w["Hq"], w["Hkv"], w["S"], w["D"]
+    var = attn.variant_select(B, Hq, Hkv, S, S, D, 1 if w["causal"] else 0)
+    structure = var // 5
+    n_qb = -(-S // 128)
+    heads = B * Hq
+    if D == 256 or structure >= 2 or heads * (-(-n_qb // 2)) < sms:
+        return heads * n_qb
+    if structure == 1 and (Hq // Hkv) % 2 == 0:
+        return heads // 2 * n_qb
+    return heads * (-(-n_qb // 2))
+
+
 def launches_per_call(w, sms=148, per_cta=2048):
     """Kernel launches of one attn_fwd call: one per batch range of at most
-    sms * per_cta work items of 256 rows (the library's split of large calls)."""
-    n_qi = -(-w["S"] // 256)
-    per_b = w["Hq"] * n_qi
+    sms * per_cta work items (the library's split of large calls)."""
+    per_b = n_items(w, sms) // w["B"]
     chunk_b = max(1, (sms * per_cta) // per_b)
     return -(-w["B"] // chunk_b)
 
@@ -305,14 +322,23 @@ def needs_l2_flush(w):
     return input_bytes(w) <= 2 * L2_BYTES
 
 
-def workload_config(w, name, n):
+INPUTS = {
+    "normal": (1.0, "Q,K,V iid N(0,1) fp16, seeded per rank"),
+    # the stress sweep's recipe: logits with std 16 make the softmax peaked, so
+    # most rows' outputs follow single values of V and most work items meet
+    # the exact pass's |O| threshold
+    "stress": (4.0, "Q,K iid N(0,4^2), V iid N(0,1) fp16 (logit std 16), seeded per rank"),
+}
+
+
+def workload_config(w, name, n, inputs="normal"):
     return {"workload": name, "B_per_gpu": w["B"], "Hq": w["Hq"], "Hkv": w["Hkv"], "S": w["S"],
             "D": w["D"], "causal": w["causal"], "global_batch": w["B"] * n,
             "parallelism": "replicas%d" % n if n > 1 else "single",
             "l2": ("L2 flushed (256 MiB written) between timed launches; time = sum of "
                    "per-launch device times" if needs_l2_flush(w) else
                    "inputs larger than L2 (no flush needed)"),
-            "inputs": "Q,K,V iid N(0,1) fp16, seeded per rank"}
+            "inputs": INPUTS[inputs][1]}
 
 
 # --------------------------------------------------------------------------- GPU arm
@@ -330,7 +356,8 @@ def run_gpu(args, w, name):
                                 device_id=dev)
     attn.load()
     B, Hq, Hkv, S, D, causal = w["B"], w["Hq"], w["Hkv"], w["S"], w["D"], w["causal"]
-    q, k, v = make_qkv(B, Hq, Hkv, S, D, seed=rank_seed(0, rank), device=dev)
+    q, k, v = make_qkv(B, Hq, Hkv, S, D, seed=rank_seed(0, rank), qk_std=INPUTS[args.inputs][0],
+                       device=dev)
     o = torch.empty_like(q)
     lse = torch.empty((B, Hq, S), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
@@ -375,7 +402,7 @@ def run_gpu(args, w, name):
     launch_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     total_ms = sum(launch_ms) if flush is not None else t_all0.elapsed_time(t_all1)
     del flush
-    st, site = attn.device_status()
+    st, site, exact_items = attn.device_status_ex()
     if st != attn.ATTN_OK:
         raise RuntimeError("device status %d at site %#x in the timed region" % (st, site))
     total_ms = reduce_max(total_ms, dev)
@@ -442,8 +469,12 @@ def run_gpu(args, w, name):
             "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f16",
-            "data": "synthetic", "config": workload_config(w, name, world),
+            "data": "synthetic", "config": workload_config(w, name, world, args.inputs),
             "e2e": e2e, "roofline": roofline, "cpu_baseline": cpu, "clocks": clocks,
+            "exact_pass": {"items_per_step": exact_items / args.steps,
+                           "items_per_step_of": n_items(w),
+                           "note": "work items recomputed with hi+lo P because a row's "
+                                   "max|O| reached the threshold (rank 0)"},
             "gpu_launches": launches_per_call(w) * args.steps,
             "pct_of_nominal_fp16_peak": 100.0 * value / world / NOMINAL_DENSE_FP16_TFLOPS,
         }
@@ -583,6 +614,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="llama3-8b-s8192-b64", choices=sorted(WORKLOADS))
     ap.add_argument("--e2e-steps", type=int, default=8)
+    ap.add_argument("--inputs", choices=sorted(INPUTS), default="normal",
+                    help="input distribution: normal (N(0,1)) or stress (logit std 16)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
