@@ -42,6 +42,9 @@ PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "attn_fwd_llama3-8b-s8192-b64.m
 KERNEL_SOURCES = [os.path.join(ROOT, "dnn_compiler_pipelining_b200", "csrc", f)
                   for f in ("attn_fwd_sm100.cuh", "ptx_sm100.cuh", "attn_api.cu",
                             "variant_table.inc")]
+LAYER_PROFILE = os.path.join(ROOT, "profiles", "decoder_layer_llama3-8b-s8192-b1.md")
+GEMM_SOURCES = [os.path.join(ROOT, "dnn_compiler_pipelining_b200", "csrc", f)
+                for f in ("gemm_sm100.cuh", "ptx_sm100.cuh", "decoder_api.cu")]
 
 
 def attn_flops(B, Hq, S, D, causal):
@@ -106,11 +109,11 @@ def code_tokens(text):
     return " ".join("".join(out).split())
 
 
-def kernel_source_hash():
+def kernel_source_hash(sources=None):
     """Hash of the code (comments and layout ignored) of the sources that
     make the timed kernel; profiles/ records it next to the counters."""
     h = hashlib.sha256()
-    for f in KERNEL_SOURCES:
+    for f in (sources or KERNEL_SOURCES):
         with open(f) as fh:
             h.update(code_tokens(fh.read()).encode())
     return h.hexdigest()[:16]
@@ -126,16 +129,16 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def profiled_traffic():
-    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+def profiled_traffic(path=PROFILE_SUMMARY, sources=None):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
     the current kernel source; else None."""
     try:
-        text = open(PROFILE_SUMMARY).read()
+        text = open(path).read()
     except OSError:
         return None
     m_h = re.search(r"kernel_source_sha256_16:\s*([0-9a-f]{16})", text)
     m_t = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
-    if not (m_h and m_t) or m_h.group(1) != kernel_source_hash():
+    if not (m_h and m_t) or m_h.group(1) != kernel_source_hash(sources):
         return None
     return float(m_t.group(1))
 
@@ -585,7 +588,11 @@ def run_layer(args):
                    "hidden": hidden, "Hq": Hq, "Hkv": Hkv, "D": D, "inter": inter,
                    "causal": True, "l2": "activations and weights larger than L2"},
         "roofline": {"bound": "tensor", "achieved": value, "peak": peak, "unit": "TFLOP/s",
-                     "frac": value / peak, "traffic": None,
+                     "frac": value / peak,
+                     "traffic": (profiled_traffic(LAYER_PROFILE, GEMM_SOURCES)
+                                 if args.layer == "llama3-8b" and S == 8192 and B == 1 else None),
+                     "traffic_of": "the gate/up GEMM (the layer's largest kernel), one launch, "
+                                   "DRAM read + write from the committed ncu capture",
                      "peak_source": "%s bf16 dense GEMM, sustained (the layer runs for several ms "
                                     "per step, back to back)" % src,
                      "algorithmic_flops_per_step": flops},

@@ -60,11 +60,14 @@ def silu(a):
 
 
 def decoder_layer(x, w_attn_norm, w_qkv, w_o, w_mlp_norm, w_gate_up, w_down, Hq, Hkv, D, eps,
-                  theta, round_fp16=True):
+                  theta, round_fp16=True, intermediates=None):
     """One LLaMA3 decoder layer.  x [B, S, hidden]; weights as the C ABI lays
     them out (w_qkv [(Hq + 2 Hkv) D, hidden] with query, key, value heads in
     that order; w_o [hidden, Hq D]; w_gate_up [2 I, hidden] gate rows then up
-    rows; w_down [hidden, I]).  Returns y [B, S, hidden] in fp64."""
+    rows; w_down [hidden, I]).  Returns y [B, S, hidden] in fp64.  A dict
+    passed as ``intermediates`` receives the stored tensors (o_tok: the
+    attention output per token [B, S, Hq D], h, g) for error budgets; the
+    arithmetic is the same either way."""
     r = f16 if round_fp16 else (lambda a: np.asarray(a, dtype=np.float64))
     x = np.asarray(x, dtype=np.float64)
     B, S, _ = x.shape
@@ -85,4 +88,6 @@ def decoder_layer(x, w_attn_norm, w_qkv, w_o, w_mlp_norm, w_gate_up, w_down, Hq,
     n2 = r(rmsnorm(h, w_mlp_norm, eps))
     gu = r(n2 @ np.asarray(w_gate_up, dtype=np.float64).T)
     g = r(silu(gu[..., :inter]) * gu[..., inter:])
+    if intermediates is not None:
+        intermediates.update(o_tok=o_tok, h=h, g=g)
     return r(h + g @ np.asarray(w_down, dtype=np.float64).T)
