@@ -48,10 +48,11 @@
 // max grows by more than 2^kRescaleLog2 (exact: O and l share the
 // reference).  The output is rounded to fp16, whose half-ulp for |O| >= 4 is
 // 1.95e-3, so rows there need more than fp16 weights can give: the epilogue
-// marks every item with a row max|O| >= kRedoThreshold in a shared-memory
-// bit set, and after its last item the CTA recomputes the marked ones with P
-// split as hi + lo fp16 (about 22-bit weights, one extra PV MMA per block):
-// the exact pass, in the same launch.
+// marks every 128-row tile with a row max|O| >= kRedoThreshold in a
+// shared-memory bit set, and after its last item the CTA recomputes the
+// marked tiles (an item whose other tile is unmarked runs with that tile
+// left out) with P split as hi + lo fp16 (about 22-bit weights, one extra
+// PV MMA per block): the exact pass, in the same launch.
 #pragma once
 
 #include <cuda_fp16.h>
@@ -70,7 +71,8 @@ constexpr float kRescaleLog2 = 8.0f;
 constexpr float kRedoThreshold = 3.98f;
 constexpr float kLn2 = 0.69314718055994531f;
 // Items of one CTA in one launch are at most 32 * kRedoWords (the exact-pass
-// bit set); the host splits larger calls.
+// bit sets: one bit per item, or per tile in the two-tile kernel); the host
+// splits larger calls.
 constexpr int kRedoWords = 64;
 constexpr int kMaxItemsPerCta = 32 * kRedoWords;
 
@@ -184,7 +186,7 @@ struct SharedFwdT {
   uint8_t v[kStagesV][tile_bytes<kD>()];
   float stat_m[2][kBlockM];  // [tile][row], handed from softmax to epilogue
   float stat_l[2][kBlockM];
-  uint32_t redo_bits[kRedoWords];  // bit k: item k of this CTA needs the exact pass
+  uint32_t redo_bits[2 * kRedoWords];  // bit 2k + x: tile x of item k needs the exact pass
   uint64_t q_full[2], q_empty[2];
   uint64_t k_full[kStagesK], k_empty[kStagesK], v_full[kStagesV], v_empty[kStagesV];
   uint64_t s_full[2], p_full[2], o_done[2], o_free[2], stats_ready[2], stats_free[2];
@@ -269,9 +271,28 @@ struct ItemWalk {
   __device__ __forceinline__ ItemWalk() : k(0), n_fast(-1), exact(false) {}
 };
 
+// The tiles of item k (bit x: tile x) that the exact pass recomputes.
 template <int kD>
-__device__ __forceinline__ bool redo_marked(const SharedFwdT<kD>* sm, int k) {
-  return (sm->redo_bits[k >> 5] >> (k & 31)) & 1u;
+__device__ __forceinline__ uint32_t redo_marked(const SharedFwdT<kD>* sm, int k) {
+  return (sm->redo_bits[(2 * k) >> 5] >> ((2 * k) & 31)) & 3u;
+}
+
+// An item of the exact pass keeps only its marked tiles.
+__device__ __forceinline__ Item exact_tiles(Item it, uint32_t tiles) {
+#pragma unroll
+  for (int x = 0; x < 2; ++x)
+    if (!((tiles >> x) & 1u)) it.n_kv[x] = 0;
+  it.n_blocks = max(it.n_kv[0], it.n_kv[1]);
+  return it;
+}
+
+// decode_item, restricted in the exact pass to the marked tiles of the item
+// the walk just returned.
+template <int kD>
+__device__ __forceinline__ Item walk_item(const FwdParams& p, const SharedFwdT<kD>* sm,
+                                          const ItemWalk& w, int item) {
+  const Item it = decode_item(p, item);
+  return w.exact ? exact_tiles(it, redo_marked(sm, w.k - 1)) : it;
 }
 
 // Next item of the walk, or -1 at the end.  At the switch from the fast pass
@@ -379,7 +400,7 @@ __device__ __forceinline__ void producer_role(SharedFwdT<kD>* sm, const FwdParam
   ItemWalk w;
   int item;
   while (ok && (item = walk_next(w, p, sm, abort, ok, kSiteProducerRedo)) >= 0) {
-    const Item it = decode_item(p, item);
+    const Item it = walk_item(p, sm, w, item);
     if (!is_v) {
 #pragma unroll
       for (int x = 0; x < 2; ++x) {
@@ -418,9 +439,10 @@ __device__ __forceinline__ void producer_role(SharedFwdT<kD>* sm, const FwdParam
     }
   }
   if (!is_v && ok && w.exact) {
-    // count this CTA's exact-pass items for the call's status block
+    // count this CTA's exact-pass items (any tile marked) for the status block
     int n = 0;
-    for (int i = 0; i < kRedoWords; ++i) n += __popc(sm->redo_bits[i]);
+    for (int i = 0; i < 2 * kRedoWords; ++i)
+      n += __popc((sm->redo_bits[i] | (sm->redo_bits[i] >> 1)) & 0x55555555u);
     if (n) atomicAdd(&p.status[2], static_cast<unsigned int>(n));
   }
   if (*abort) {
@@ -452,7 +474,7 @@ __device__ __forceinline__ void mma_role(SharedFwdT<kD>* sm, const FwdParams& p,
   ItemWalk w;
   int item;
   while (ok && (item = walk_next<kD, true>(w, p, sm, abort, ok, kSiteMmaRedo)) >= 0) {
-    const Item it = decode_item(p, item);
+    const Item it = walk_item(p, sm, w, item);
     const bool hilo = w.exact;
     const int n_b = it.n_blocks;
     for (int j = 0; ok && j <= n_b; ++j) {
@@ -520,12 +542,12 @@ __device__ __forceinline__ void mma_role(SharedFwdT<kD>* sm, const FwdParams& p,
 }
 
 // Epilogue of one item (warps 8-11; thread r owns row r of both tiles):
-// O / l -> fp16 and LSE.  Returns false if a wait gave up; `flag` tells
-// whether a stored row has max|O| >= kRedoThreshold.
+// O / l -> fp16 and LSE.  Returns false if a wait gave up; bit x of `flag`
+// is set when a stored row of tile x has max|O| >= kRedoThreshold.
 template <int kD>
 __device__ __forceinline__ bool epilogue_item(SharedFwdT<kD>* sm, const FwdParams& p,
                                               uint32_t lane_base, int r, int lane, const Item& it,
-                                              int (&ecnt)[2], bool& flag, volatile int* abort) {
+                                              int (&ecnt)[2], uint32_t& flag, volatile int* abort) {
   const uint64_t to = p.timeout_ns;
   bool ok = true;
 #pragma unroll
@@ -581,7 +603,7 @@ __device__ __forceinline__ bool epilogue_item(SharedFwdT<kD>* sm, const FwdParam
     __syncwarp();
     if (lane == 0) mbar_arrive(smem_addr(&sm->o_free[x]));
     if (valid) p.lse[row] = (m_use + log2f(l)) * kLn2;
-    flag |= valid && omax >= kRedoThreshold;
+    if (valid && omax >= kRedoThreshold) flag |= 1u << x;
   }
   return ok;
 }
@@ -599,10 +621,10 @@ __device__ __forceinline__ void epilogue_role(SharedFwdT<kD>* sm, const FwdParam
   bool ok = true;
   int k = 0;
   for (int item; ok && (item = seq_item(p, k)) >= 0; ++k) {
-    bool flag = false;
+    uint32_t flag = 0;
     ok = epilogue_item(sm, p, lane_base, r, lane, decode_item(p, item), ecnt, flag, abort);
-    if (ok && __any_sync(0xffffffffu, flag) && lane == 0)
-      atomicOr(&sm->redo_bits[k >> 5], 1u << (k & 31));
+    const uint32_t tiles = __reduce_or_sync(0xffffffffu, flag);
+    if (ok && tiles && lane == 0) atomicOr(&sm->redo_bits[(2 * k) >> 5], tiles << ((2 * k) & 31));
   }
   // every fast-pass item is marked or not: release the others (also when
   // this warp gave up, so that no role waits for the marks forever)
@@ -613,10 +635,11 @@ __device__ __forceinline__ void epilogue_role(SharedFwdT<kD>* sm, const FwdParam
                  kSiteEpilogueRedo);
   if (!__all_sync(0xffffffffu, ok)) return;
   for (int kk = 0; ok && kk < k; ++kk) {
-    if (!redo_marked(sm, kk)) continue;
-    bool flag = false;
-    ok = epilogue_item(sm, p, lane_base, r, lane, decode_item(p, seq_item(p, kk)), ecnt, flag,
-                       abort);
+    const uint32_t tiles = redo_marked(sm, kk);
+    if (!tiles) continue;
+    uint32_t flag = 0;
+    ok = epilogue_item(sm, p, lane_base, r, lane, exact_tiles(decode_item(p, seq_item(p, kk)), tiles),
+                       ecnt, flag, abort);
   }
 }
 
@@ -760,7 +783,7 @@ __device__ __forceinline__ void softmax_role(SharedFwdT<kD>* sm, const FwdParams
   ItemWalk w;
   int item;
   while (ok && (item = walk_next(w, p, sm, abort, ok, kSiteSoftmaxRedo)) >= 0) {
-    const Item it = decode_item(p, item);
+    const Item it = walk_item(p, sm, w, item);
     const int n_x = x ? it.n_kv[1] : it.n_kv[0];
     if (n_x == 0) continue;
     // the last key this row sees: row + off (causal), and never past Sk (a
@@ -832,7 +855,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(smem_addr(&sm->v_empty[s]), 1);
     }
     mbar_init(smem_addr(&sm->redo_ready), 4);
-    for (int i = 0; i < kRedoWords; ++i) sm->redo_bits[i] = 0;
+    for (int i = 0; i < 2 * kRedoWords; ++i) sm->redo_bits[i] = 0;
     sm->abort = 0;
     fence_mbar_init();
   }
