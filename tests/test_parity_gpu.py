@@ -395,6 +395,49 @@ def test_large_outputs_every_item_exact():
     parity.full_check(1, 2, 1, 256, 128, True, seed=26)
 
 
+@pytest.mark.parametrize("large_keys", ["first", "second"])
+def test_exact_pass_one_tile_of_an_item(large_keys):
+    """Items of 256 rows (the ping-pong kernel, variant 0, with enough heads
+    for two-tile items) where only one 128-row tile has |O| >= 4.  V is large
+    (|v| in [4, 6]) only on keys 0-127 ("first": the first rows of tile A
+    follow those values, tile B averages them with small ones under diffuse
+    logits) or only on keys 128-255 ("second": peaked logits, so rows of tile
+    B follow single large values, while tile A never sees those keys).  The
+    exact pass runs the marked tile alone; every row must match the oracle,
+    and the call counts each item with a marked tile once."""
+    B, Hq, Hkv, S, D = 8, 32, 8, 256, 128   # one 256-row item per head, 256 items
+    qk_std = 0.5 if large_keys == "first" else 4.0
+    q, k, v = make_qkv(B, Hq, Hkv, S, D, seed=31, qk_std=qk_std, device="cuda")
+    big = _large_v(B, Hkv, S, D, 32)
+    small = (v.float() * 0.01).half()
+    keys = torch.arange(S, device="cuda").view(1, 1, S, 1)
+    in_large = keys < 128 if large_keys == "first" else keys >= 128
+    v = torch.where(in_large, big, small).contiguous()
+    attn.device_status_ex()  # clear
+    o = torch.full_like(q, float("nan"))
+    lse = torch.full((B, Hq, S), float("nan"), dtype=torch.float32, device="cuda")
+    attn.attn_fwd_variant(q, k, v, True, 0, o=o, lse=lse)
+    st, site, n_exact = attn.device_status_ex()
+    assert st == attn.ATTN_OK, "device status %d at site %#x" % (st, site)
+    import oracle
+    o_ref, lse_ref = oracle.attention(q.cpu().double().numpy(), k.cpu().double().numpy(),
+                                      v.cpu().double().numpy(), True)
+    row_max = np.abs(o_ref).max(axis=-1)                      # [B, Hq, S]
+
+    def marked(thr):
+        return (row_max >= thr).reshape(B, Hq, 2, 128).any(axis=-1)   # [B, Hq, tile]
+    # the kernel applies the threshold to its own O; rows within 0.01 of it
+    # may go either way
+    surely, maybe = marked(3.98 + 0.01), marked(3.98 - 0.01)
+    if large_keys == "first":
+        assert surely[..., 0].all() and not maybe[..., 1].any()
+    else:
+        assert surely[..., 1].any() and not maybe[..., 0].any()
+    assert int(surely.any(axis=-1).sum()) <= n_exact <= int(maybe.any(axis=-1).sum()), n_exact
+    parity.assert_close(o.cpu().double().numpy(), o_ref, lse.cpu().double().numpy(), lse_ref,
+                        "one tile marked (%s)" % large_keys)
+
+
 def test_exact_pass_only_where_needed():
     """N(0,1) inputs at a long sequence: outputs average many V rows, so only
     the first rows of a head can reach |O| >= 3.98 -- few items, all of them
