@@ -193,8 +193,9 @@ attn_status attn_device_status(void* stream, uint32_t* site);
 
 /*
  * attn_device_status_ex -- attn_device_status, plus `exact_items` (if not
- * NULL): the number of work items the kernels on `stream` recomputed with
- * two-part probabilities since the last read.
+ * NULL): the number of work items (256 or 128 query rows of a head) of which
+ * the kernels on `stream` recomputed at least one 128-row tile with two-part
+ * probabilities since the last read.
  */
 attn_status attn_device_status_ex(void* stream, uint32_t* site, uint64_t* exact_items);
 
