@@ -28,18 +28,6 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
   return t;
 }
 
-// One lane of a converged warp (the same lane every time): 1 there, 0 in the
-// other lanes.
-__device__ __forceinline__ uint32_t elect_one() {
-  uint32_t e;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "elect.sync _|p, 0xffffffff;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(e));
-  return e;
-}
-
 // Register reallocation between warpgroups (every warp of a warpgroup
 // executes the same one).
 template <int kRegs>
