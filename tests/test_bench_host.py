@@ -1,5 +1,7 @@
 """bench.py host logic on the CPU: the kernel-source hash that ties the
-committed ncu counters to the code, FLOP counts, and the L2-flush rule."""
+committed ncu counters to the code, FLOP counts, the L2-flush rule, the work
+items and launches per call that follow the library's variant table, and the
+stress-input recipe."""
 import os
 import sys
 
@@ -37,3 +39,48 @@ def test_flop_counts():
     per_token = 2.0 * 4096 * (48 * 128 + 32 * 128 + 3 * 14336)
     assert bench.layer_flops(1, 1, 4096, 32, 8, 128, 14336) == per_token + \
         bench.attn_flops(1, 32, 1, 128, True)
+
+
+def test_l2_flush_rule():
+    from dnn_compiler_pipelining_b200.inputs import WORKLOADS
+    # Q + K + V of the small single-batch workloads fit in twice the L2: flushed
+    assert bench.needs_l2_flush(WORKLOADS["llama3-8b-s512-b1"])
+    assert bench.needs_l2_flush(WORKLOADS["llama3-8b-s8192-b1"])
+    # the batched workloads stream far more than the L2 holds
+    assert not bench.needs_l2_flush(WORKLOADS["llama3-8b-s8192-b64"])
+    assert not bench.needs_l2_flush(WORKLOADS["llama3-8b-s2048-b64"])
+
+
+def test_items_and_launches_follow_the_variant_table():
+    from dnn_compiler_pipelining_b200.build import build
+    build()
+    from dnn_compiler_pipelining_b200.inputs import WORKLOADS
+    w = WORKLOADS["llama3-8b-s8192-b64"]            # variant 0: 256-row items
+    assert bench.n_items(w) == 64 * 32 * 32
+    assert bench.launches_per_call(w) == 1
+    w = WORKLOADS["llama3-8b-s512-b1"]              # double-buffered kernel: 128-row items
+    assert bench.n_items(w) == 32 * 4
+    w = dict(B=1, Hq=32, Hkv=8, S=8192, D=128, causal=True)  # 256-row items fill the SMs
+    assert bench.n_items(w) == 32 * 32
+    w = dict(B=1, Hq=8, Hkv=8, S=2048, D=128, causal=False)  # too few 256-row items: 128
+    assert bench.n_items(w) == 8 * 16
+    # more items than one launch's per-CTA bit set holds: split over batch ranges
+    w = dict(B=4096, Hq=32, Hkv=8, S=8192, D=128, causal=True)
+    assert bench.launches_per_call(w) == -(-4096 * 32 * 32 // (148 * 2048 // (32 * 32) * 32 * 32))
+
+
+def test_stress_inputs_recipe():
+    assert bench.INPUTS["normal"][0] == 1.0 and bench.INPUTS["stress"][0] == 4.0
+    cfg = bench.workload_config(dict(B=1, Hq=32, Hkv=8, S=512, D=128, causal=True), "x", 1,
+                                "stress")
+    assert "N(0,4^2)" in cfg["inputs"]
+
+
+def test_profiled_traffic_needs_matching_source(tmp_path, monkeypatch):
+    prof = tmp_path / "p.md"
+    prof.write_text("kernel_source_sha256_16: %s\ndram_bytes_per_launch: 1.5e9\n"
+                    % bench.kernel_source_hash())
+    assert bench.profiled_traffic(str(prof)) == 1.5e9
+    prof.write_text("kernel_source_sha256_16: 0123456789abcdef\ndram_bytes_per_launch: 1.5e9\n")
+    assert bench.profiled_traffic(str(prof)) is None
+    assert bench.profiled_traffic(str(tmp_path / "missing.md")) is None
