@@ -57,7 +57,7 @@ typedef enum attn_status {
   ATTN_ERR_NULL = 1,           /* a required pointer is NULL */
   ATTN_ERR_SHAPE = 2,          /* B,Hq,Hkv,S < 1, Hq % Hkv != 0, or a size overflows */
   ATTN_ERR_ALIGN = 3,          /* q, k, v, o not 16-byte aligned, or lse not 4-byte aligned */
-  ATTN_ERR_UNSUPPORTED = 4,    /* D not 64 or 128, or not an sm_100 device */
+  ATTN_ERR_UNSUPPORTED = 4,    /* D not 64, 128 or 256, or not an sm_100 device */
   ATTN_ERR_CUDA = 5,           /* a CUDA runtime / driver call failed */
   ATTN_ERR_DEVICE_TIMEOUT = 6, /* a kernel wait ran out; results are invalid */
   ATTN_ERR_WORKSPACE = 7,      /* the device workspace given is too small */
@@ -71,7 +71,7 @@ typedef enum attn_status {
  *   k, v: device, fp16 [B, Hkv, S, D], 16-byte aligned, read only.
  *   o   : device, fp16 [B, Hq, S, D], 16-byte aligned, written.
  *   lse : device, fp32 [B, Hq, S], 4-byte aligned, written (must not be NULL).
- *   B, Hq, Hkv, S, D: sizes; Hq % Hkv == 0; D == 64 or 128; any S >= 1 (a
+ *   B, Hq, Hkv, S, D: sizes; Hq % Hkv == 0; D == 64, 128 or 256; any S >= 1 (a
  *   last block of fewer than 128 rows is computed with the keys past S
  *   masked).
  *   causal: nonzero for the causal mask j <= i (square, Sq == Sk == S).
@@ -79,11 +79,12 @@ typedef enum attn_status {
  * Returns ATTN_OK once the kernel is enqueued; errors as listed above.  The
  * outputs must not overlap the inputs.  One kernel runs on `stream` (a call
  * with more than 2048 work items per SM is split into launches over batch
- * ranges).  Each CTA of it computes its work items (256 or 128 query rows of
- * one head) with fp16 probabilities, then recomputes, with the
- * probabilities split into two fp16 parts, the items that have a row with
- * max|O| >= 3.98, where fp16 output rounding leaves almost no error budget;
- * attn_device_status_ex() reports how many items that were.
+ * ranges).  Each CTA of it computes its work items (256 query rows: two
+ * 128-row tiles of one head or of two heads of a group; or 128 rows) with
+ * fp16 probabilities, then recomputes, with the probabilities split into two
+ * fp16 parts, the 128-row tiles that have a row with max|O| >= 3.98, where
+ * fp16 output rounding leaves almost no error budget;
+ * attn_device_status_ex() reports how many items had such a tile.
  */
 attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
                      int B, int Hq, int Hkv, int S, int D, int causal, void* stream);
