@@ -241,6 +241,20 @@ def test_stress_sweep(pt):
     torch.cuda.empty_cache()
 
 
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("B,Hq,Hkv,S", [(8, 24, 8, 1000), (4, 32, 8, 1100), (2, 24, 8, 6000)])
+def test_default_head_pairs(B, Hq, Hkv, S, causal):
+    """Calls the table sends to the head-pair ping-pong (enough heads for
+    two-tile items): an even group pairs the same rows of two heads, an odd
+    one (24 / 8 = 3) falls back to row pairs; ragged S in both."""
+    from tests.test_variants import table_rules, expected_variant
+    var = attn.variant_select(B, Hq, Hkv, S, S, 128, 1 if causal else 0)
+    assert var == expected_variant(table_rules(), 128, 1 if causal else 0, S)
+    q, k, v = make_qkv(B, Hq, Hkv, S, 128, seed=41, device="cuda")
+    o, lse = parity.run_gpu(q, k, v, causal)
+    parity.sampled_check(q, k, v, o, lse, causal, n_random=384, seed=42)
+
+
 def test_deterministic():
     q, k, v = make_qkv(2, 8, 2, 1024, 128, seed=3, device="cuda")
     o1, l1 = parity.run_gpu(q, k, v, True)
