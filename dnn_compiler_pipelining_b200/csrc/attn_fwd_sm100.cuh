@@ -70,6 +70,7 @@ constexpr uint32_t kPanelBytes = 16384;  // 128 rows x 64 fp16: one 128-byte swi
 constexpr float kRescaleLog2 = 8.0f;
 constexpr float kRedoThreshold = 3.98f;
 constexpr float kLn2 = 0.69314718055994531f;
+constexpr float kLog2e = 1.44269504088896341f;
 // Items of one CTA in one launch are at most 32 * kRedoWords (the exact-pass
 // bit sets: one bit per item, or per tile in the two-tile kernel); the host
 // splits larger calls.
@@ -768,6 +769,67 @@ __device__ __forceinline__ bool softmax_item(SharedFwdT<kD>* sm, const FwdParams
   return true;
 }
 
+// The key blocks of one item in the exact pass.  The fast pass has already
+// stored the row's LSE = ln 2 * (m + log2 l) in log2 units m + log2 l, which
+// bounds every scaled logit of the row from above: l sums the weights
+// against m, the largest of them among them, even when a lazy rescale left m
+// below the row max.  With m_ref = that bound - kRescaleLog2, the weights
+// p = 2^(s * scale - m_ref) stay <= 2^kRescaleLog2 (the fast pass's range,
+// well inside fp16 and away from its subnormals) with no running max and no
+// rescale of O.  P goes to the PV MMAs as hi + lo fp16 (hi over columns
+// [0, 64), lo over [64, 128)); l sums the fp32 p.  Returns false if a wait
+// gave up.
+template <int kD>
+__device__ __forceinline__ bool softmax_item_exact(SharedFwdT<kD>* sm, const FwdParams& p, int x,
+                                                   uint32_t s_t, int n_x, int key_lim,
+                                                   int j_mask, int lane, int& scnt, float m_ref,
+                                                   float& l, volatile int* abort) {
+  const uint64_t to = p.timeout_ns;
+  const float sc = p.scale_log2;
+  const float neg_m = -m_ref;
+  l = 0.f;
+  for (int j = 0; j < n_x; ++j, ++scnt) {
+    bool ok = mbar_wait(smem_addr(&sm->s_full[x]), scnt & 1, abort, to, p.status, kSiteSoftmaxS);
+    if (!__all_sync(0xffffffffu, ok)) return false;
+    tc_fence_after();
+    // the whole row of S first: P's low parts go over columns [64, 128)
+    uint32_t u[128];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) tmem_ld32(s_t + c * 32, &u[c * 32]);
+    tmem_wait_ld();
+#pragma unroll
+    for (int c = 0; c < 4; ++c) reg_dep32(&u[c * 32]);
+    if (j >= j_mask) {
+      const int lim = key_lim - j * kBlockN;
+#pragma unroll
+      for (int c = 0; c < 128; ++c)
+        if (c > lim) u[c] = 0xff800000u;  // -inf
+    }
+    float lp[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      uint32_t ph[8], pl[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float p0 = ex2_approx(fmaf(__uint_as_float(u[c * 16 + 2 * i]), sc, neg_m));
+        const float p1 = ex2_approx(fmaf(__uint_as_float(u[c * 16 + 2 * i + 1]), sc, neg_m));
+        ph[i] = pack_half2(p0, p1);
+        const float2 hh = __half22float2(*reinterpret_cast<const __half2*>(&ph[i]));
+        pl[i] = pack_half2(p0 - hh.x, p1 - hh.y);
+        lp[i & 3] += p0 + p1;
+      }
+      tmem_st8(s_t + c * 8, ph);
+      tmem_st8(s_t + 64 + c * 8, pl);
+    }
+    l += (lp[0] + lp[1]) + (lp[2] + lp[3]);
+    tmem_wait_st();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(smem_addr(&sm->p_full[x]));
+  }
+  return true;
+}
+
 // Softmax of tile x (warps 4x..4x+3).
 template <int kD, int kEmu>
 __device__ __forceinline__ void softmax_role(SharedFwdT<kD>* sm, const FwdParams& p, uint32_t tmem,
@@ -795,10 +857,19 @@ __device__ __forceinline__ void softmax_role(SharedFwdT<kD>* sm, const FwdParams
     // lane of the warp has keys to mask
     const int j_mask = (__shfl_sync(0xffffffffu, key_lim, 0) + 1) / kBlockN;
     float m_use, l;
-    ok = w.exact ? softmax_item<kD, kEmu, true>(sm, p, x, s_t, o_t, n_x, key_lim, j_mask, lane,
-                                                 scnt, m_use, l, abort)
-                 : softmax_item<kD, kEmu, false>(sm, p, x, s_t, o_t, n_x, key_lim, j_mask, lane,
-                                                  scnt, m_use, l, abort);
+    if (w.exact) {
+      // the fast pass stored this row's LSE (rows past S: not stored, not
+      // needed, any finite reference does)
+      const int hq = it.hq + x * it.dhq;
+      const float lse = i_row < p.S ? p.lse[(static_cast<size_t>(it.b) * p.Hq + hq) * p.S + i_row]
+                                    : 0.f;
+      m_use = lse * kLog2e - kRescaleLog2;
+      ok = softmax_item_exact<kD>(sm, p, x, s_t, n_x, key_lim, j_mask, lane, scnt, m_use, l,
+                                  abort);
+    } else {
+      ok = softmax_item<kD, kEmu, false>(sm, p, x, s_t, o_t, n_x, key_lim, j_mask, lane, scnt,
+                                         m_use, l, abort);
+    }
     if (!ok) break;
     // the epilogue must have read this tile's previous statistics
     ok = acnt == 0 || mbar_wait(smem_addr(&sm->stats_free[x]), (acnt - 1) & 1, abort,
