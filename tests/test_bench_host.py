@@ -84,3 +84,13 @@ def test_profiled_traffic_needs_matching_source(tmp_path, monkeypatch):
     prof.write_text("kernel_source_sha256_16: 0123456789abcdef\ndram_bytes_per_launch: 1.5e9\n")
     assert bench.profiled_traffic(str(prof)) is None
     assert bench.profiled_traffic(str(tmp_path / "missing.md")) is None
+
+
+def test_traffic_only_for_the_profiled_case(monkeypatch):
+    monkeypatch.setattr(bench, "profiled_traffic", lambda *a, **k: 7.0e9)
+    assert bench.attn_traffic(*bench.PROFILED_CASE) == 7.0e9
+    from dnn_compiler_pipelining_b200.inputs import WORKLOADS
+    assert bench.PROFILED_CASE[0] in WORKLOADS
+    assert bench.attn_traffic(bench.PROFILED_CASE[0], "stress") is None
+    other = next(n for n in WORKLOADS if n != bench.PROFILED_CASE[0])
+    assert bench.attn_traffic(other, "normal") is None
