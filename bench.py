@@ -145,6 +145,21 @@ def profiled_traffic(path=PROFILE_SUMMARY, sources=None):
     return float(m_t.group(1))
 
 
+def algorithmic_bytes(B, Hq, Hkv, S, D):
+    """Bytes one attention call must move at the least: Q, K, V read once (fp16),
+    O (fp16) and LSE (fp32) written once."""
+    return 2 * S * D * (2 * B * Hq + 2 * B * Hkv) + 4 * B * Hq * S
+
+
+def hbm_figure(nbytes, launch_ms, peak_gbs, peak_src):
+    """The call's algorithmic bytes per second against the measured copy
+    bandwidth: the bound that matters where the launch is too short for the
+    tensor pipe to dominate (a single short sequence)."""
+    gbs = nbytes / (launch_ms * 1e-3) / 1e9
+    return {"algorithmic_bytes_per_launch": nbytes, "achieved_gbs": gbs, "peak_gbs": peak_gbs,
+            "frac": gbs / peak_gbs, "peak_source": "%s HBM copy bandwidth" % peak_src}
+
+
 def attn_traffic(workload, inputs):
     """The fused pass's DRAM bytes per launch for `workload` on `inputs`: the
     committed capture's figure for the case it was taken on, None for any
@@ -466,8 +481,11 @@ def run_gpu(args, w, name):
                 "frac_of_sustained_peak": achieved / peak_sus,
                 "frac_of_nominal_2250": achieved / NOMINAL_DENSE_FP16_TFLOPS,
                 "algorithmic_flops_per_launch": flops,
-                "launch_ms": {"mean": avg_launch_ms, "min": min(launch_ms),
-                              "max": max(launch_ms)}}
+                "launch_ms": {"mean": avg_launch_ms, "median": statistics.median(launch_ms),
+                              "min": min(launch_ms), "max": max(launch_ms)},
+                "hbm": hbm_figure(algorithmic_bytes(B, Hq, Hkv, S, D), avg_launch_ms,
+                                  float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])),
+                                  src)}
 
     cpu = None
     if rank == 0 and not args.no_cpu_baseline:

@@ -94,3 +94,14 @@ def test_traffic_only_for_the_profiled_case(monkeypatch):
     assert bench.attn_traffic(bench.PROFILED_CASE[0], "stress") is None
     other = next(n for n in WORKLOADS if n != bench.PROFILED_CASE[0])
     assert bench.attn_traffic(other, "normal") is None
+
+
+def test_algorithmic_bytes_of_the_target_shape():
+    # Q and O: 64*32*8192*128 fp16 each (4 GiB); K and V: 64*8*8192*128 fp16 each
+    # (1 GiB); LSE: 64*32*8192 fp32 (64 MiB) -- 10.80 GB in all
+    n = bench.algorithmic_bytes(64, 32, 8, 8192, 128)
+    assert n == 2 * 2**32 + 2 * 2**30 + 2**26
+    assert abs(n / 1e9 - 10.80) < 0.01
+    h = bench.hbm_figure(n, 10.0, 6000.0, "measured")
+    assert abs(h["achieved_gbs"] - n / 1e-2 / 1e9) < 1e-9
+    assert abs(h["frac"] - h["achieved_gbs"] / 6000.0) < 1e-12
