@@ -327,8 +327,12 @@ attn_status launch_call(const void* q, const void* k, const void* v, void* o, fl
 // Streams of attn_fwd_host's copy / compute pipeline, created once per device
 // (non-blocking, so they do not serialize with the legacy default stream).
 constexpr int kHostChunks = 16;
+// One call at a time uses a device's pipeline (`busy`): concurrent calls would
+// share the compute stream's status block, and one could read and clear a
+// timeout that the other's kernels raised.
 struct HostPipe {
   cudaStream_t up, comp, down;
+  std::mutex busy;
 };
 HostPipe* g_host_pipe[kMaxDevices];
 std::mutex g_host_pipe_mutex;
@@ -538,6 +542,7 @@ attn_status attn_fwd_host(const void* q_h, const void* k_h, const void* v_h, voi
   // already on `stream`; `stream` waits for the last download.
   HostPipe* hp = host_pipe(dev);
   if (!hp) return ATTN_ERR_CUDA;
+  std::lock_guard<std::mutex> one_call(hp->busy);
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   const int n_chunks = B < kHostChunks ? B : kHostChunks;
   cudaEvent_t ev[1 + 2 * kHostChunks + 1];

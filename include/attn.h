@@ -173,6 +173,8 @@ size_t attn_fwd_host_workspace_bytes(int B, int Hq, int Hkv, int S, int D);
  * host buffers hold the results on ATTN_OK.  Host buffers may be pageable or
  * pinned (pinned copies run asynchronously and faster).  The library creates
  * those three streams on its first call for each device and keeps them.
+ * Concurrent calls on one device (from several host threads) run one after
+ * another, so each call's status is its own.
  *   workspace: device, >= attn_fwd_host_workspace_bytes(...) bytes, 256-byte
  *              aligned; its contents are overwritten.
  * Also returns ATTN_ERR_DEVICE_TIMEOUT if the kernel reported one.

@@ -351,6 +351,43 @@ def test_host_entry_matches_device_entry(B, Hq, Hkv, S, D, pinned):
     assert torch.equal(oh, o.cpu()) and torch.equal(lh, lse.cpu())
 
 
+def test_host_entry_concurrent_threads():
+    """Two host threads call the host-buffer entry at the same time on one device
+    (ctypes drops the GIL, and the library runs the calls one after another on
+    its pipeline streams): every call gives the device entry's bytes."""
+    import threading
+    cases = []
+    for i, (B, Hq, Hkv, S) in enumerate([(6, 4, 2, 384), (5, 8, 2, 256)]):
+        q, k, v = make_qkv(B, Hq, Hkv, S, 128, seed=70 + i, device="cuda")
+        o, lse = parity.run_gpu(q, k, v, True)
+        host = [t.cpu().pin_memory() for t in (q, k, v)]
+        oh = torch.empty_like(host[0]).pin_memory()
+        lh = torch.empty((B, Hq, S), dtype=torch.float32).pin_memory()
+        ws = torch.empty(attn.host_workspace_bytes(B, Hq, Hkv, S, 128), dtype=torch.uint8,
+                         device="cuda")
+        cases.append((host, oh, lh, ws, o.cpu(), lse.cpu()))
+    torch.cuda.synchronize()
+    errors = []
+
+    def run(c):
+        try:
+            torch.cuda.set_device(0)
+            for _ in range(3):
+                c[1].fill_(float("nan"))
+                c[2].fill_(float("nan"))
+                attn.attn_fwd_host(*c[0], c[1], c[2], True, c[3])
+                assert torch.equal(c[1], c[4]) and torch.equal(c[2], c[5])
+        except Exception as e:  # reported by the main thread
+            errors.append(e)
+
+    threads = [threading.Thread(target=run, args=(c,)) for c in cases]
+    for t in threads:
+        t.start()
+    for t in threads:
+        t.join()
+    assert not errors, errors
+
+
 def test_bounded_wait_reports_timeout():
     """A wait on an mbarrier nobody completes ends after its bound with
     ATTN_ERR_DEVICE_TIMEOUT, and the context stays usable."""
