@@ -644,10 +644,10 @@ __device__ __forceinline__ void epilogue_role(SharedFwdT<kD>* sm, const FwdParam
   }
 }
 
-// The key blocks of one item for one tile's softmax warp (thread = query row
-// = TMEM lane).  kHilo: the exact pass (P = hi + lo).  Returns false if a
-// wait gave up; m_use and l hold the row's statistics on return.
-template <int kD, int kEmu, bool kHilo>
+// The key blocks of one item in the fast pass, for one tile's softmax warp
+// (thread = query row = TMEM lane).  Returns false if a wait gave up; m_use
+// and l hold the row's statistics on return.
+template <int kD, int kEmu>
 __device__ __forceinline__ bool softmax_item(SharedFwdT<kD>* sm, const FwdParams& p, int x,
                                              uint32_t s_t, uint32_t o_t, int n_x, int key_lim,
                                              int j_mask, int lane, int& scnt, float& m_use,
@@ -715,50 +715,30 @@ __device__ __forceinline__ bool softmax_item(SharedFwdT<kD>* sm, const FwdParams
     }
     const float neg_m = -m_use;
     float lp[4] = {0.f, 0.f, 0.f, 0.f};
-    if constexpr (!kHilo) {
-      // P rounded to fp16; l sums exactly the rounded values.  In every 16
-      // columns, kEmu pairs take 2^x from the FMA-pipe polynomial and the rest
-      // from the MUFU unit.
-      const float2 sc2 = make_float2(sc, sc);
-      const float2 nm2 = make_float2(neg_m, neg_m);
+    // P rounded to fp16; l sums exactly the rounded values.  In every 16
+    // columns, kEmu pairs take 2^x from the FMA-pipe polynomial and the rest
+    // from the MUFU unit.
+    const float2 sc2 = make_float2(sc, sc);
+    const float2 nm2 = make_float2(neg_m, neg_m);
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        uint32_t ph[8];
+    for (int c = 0; c < 8; ++c) {
+      uint32_t ph[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const float2 s2 = make_float2(__uint_as_float(u[c * 16 + 2 * i]),
-                                        __uint_as_float(u[c * 16 + 2 * i + 1]));
-          const float2 x2 = __ffma2_rn(s2, sc2, nm2);
-          float2 p2;
-          if (i < kEmu) {
-            p2 = exp2_poly2(x2);
-          } else {
-            p2.x = ex2_approx(x2.x);
-            p2.y = ex2_approx(x2.y);
-          }
-          ph[i] = pack_half2(p2.x, p2.y);
-          lp[i & 3] = add_half2_f32(ph[i], lp[i & 3]);
+      for (int i = 0; i < 8; ++i) {
+        const float2 s2 = make_float2(__uint_as_float(u[c * 16 + 2 * i]),
+                                      __uint_as_float(u[c * 16 + 2 * i + 1]));
+        const float2 x2 = __ffma2_rn(s2, sc2, nm2);
+        float2 p2;
+        if (i < kEmu) {
+          p2 = exp2_poly2(x2);
+        } else {
+          p2.x = ex2_approx(x2.x);
+          p2.y = ex2_approx(x2.y);
         }
-        tmem_st8(s_t + c * 8, ph);
+        ph[i] = pack_half2(p2.x, p2.y);
+        lp[i & 3] = add_half2_f32(ph[i], lp[i & 3]);
       }
-    } else {
-      // P = hi + lo, both fp16: hi over columns [0,64), lo over [64,128); l
-      // sums the fp32 p the two parts represent
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        uint32_t ph[8], pl[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const float p0 = ex2_approx(fmaf(__uint_as_float(u[c * 16 + 2 * i]), sc, neg_m));
-          const float p1 = ex2_approx(fmaf(__uint_as_float(u[c * 16 + 2 * i + 1]), sc, neg_m));
-          ph[i] = pack_half2(p0, p1);
-          const float2 h = __half22float2(*reinterpret_cast<const __half2*>(&ph[i]));
-          pl[i] = pack_half2(p0 - h.x, p1 - h.y);
-          lp[i & 3] += p0 + p1;
-        }
-        tmem_st8(s_t + c * 8, ph);
-        tmem_st8(s_t + 64 + c * 8, pl);
-      }
+      tmem_st8(s_t + c * 8, ph);
     }
     l += (lp[0] + lp[1]) + (lp[2] + lp[3]);
     tmem_wait_st();
@@ -867,8 +847,8 @@ __device__ __forceinline__ void softmax_role(SharedFwdT<kD>* sm, const FwdParams
       ok = softmax_item_exact<kD>(sm, p, x, s_t, n_x, key_lim, j_mask, lane, scnt, m_use, l,
                                   abort);
     } else {
-      ok = softmax_item<kD, kEmu, false>(sm, p, x, s_t, o_t, n_x, key_lim, j_mask, lane, scnt,
-                                         m_use, l, abort);
+      ok = softmax_item<kD, kEmu>(sm, p, x, s_t, o_t, n_x, key_lim, j_mask, lane, scnt, m_use,
+                                  l, abort);
     }
     if (!ok) break;
     // the epilogue must have read this tile's previous statistics
