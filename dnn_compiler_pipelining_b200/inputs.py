@@ -59,10 +59,13 @@ WORKLOADS = {
     "llama3-8b-s2048-b64": dict(B=64, Hq=32, Hkv=8, S=2048, D=128, causal=True),
     "llama3-70b-s8192-b64": dict(B=64, Hq=64, Hkv=8, S=8192, D=128, causal=True),
     "llama3-8b-s8192-b64": dict(B=64, Hq=32, Hkv=8, S=8192, D=128, causal=True),
+    # the large-head case: 8B head counts at head dimension 256
+    "gqa32x8-d256-s8192-b16": dict(B=16, Hq=32, Hkv=8, S=8192, D=256, causal=True),
     # small cases of the same kernel for profiler captures (Q alone exceeds L2)
     "llama3-8b-s8192-b4": dict(B=4, Hq=32, Hkv=8, S=8192, D=128, causal=True),
     "llama3-8b-s2048-b8": dict(B=8, Hq=32, Hkv=8, S=2048, D=128, causal=True),
     "llama3-70b-s8192-b4": dict(B=4, Hq=64, Hkv=8, S=8192, D=128, causal=True),
+    "gqa32x8-d256-s8192-b2": dict(B=2, Hq=32, Hkv=8, S=8192, D=256, causal=True),
 }
 
 

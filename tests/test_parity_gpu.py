@@ -208,7 +208,8 @@ def test_llama3_8b_s512_b1_full():
 
 
 @pytest.mark.parametrize("name", ["llama3-8b-s8192-b1", "llama3-8b-s2048-b64",
-                                  "llama3-8b-s8192-b64", "llama3-70b-s8192-b64"])
+                                  "llama3-8b-s8192-b64", "llama3-70b-s8192-b64",
+                                  "gqa32x8-d256-s8192-b16"])
 def test_workload_sampled(name):
     w = WORKLOADS[name]
     q, k, v = make_qkv(w["B"], w["Hq"], w["Hkv"], w["S"], w["D"], seed=0, device="cuda")
