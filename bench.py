@@ -12,9 +12,14 @@ max over ranks.  Rank 0 prints one JSON line.
 
 Other keys: `e2e` (the same metric through the host-buffer C entry point,
 H2D and D2H copies inside the timed region), `roofline` (tensor-core bound
-against the measured burst bf16 GEMM peak: the kernel is timed on its own), `cpu_baseline` (the fp64 oracle on a
-bounded sample, timed on this host's cores), `clocks` (nvidia-smi sampled
-during the timed region), `gpu_launches`.
+against the measured burst bf16 GEMM peak: the kernel is timed on its own;
+`traffic` is the DRAM bytes per launch of the committed ncu capture, given
+only for the workload and inputs it was taken on and while the kernel
+sources match it; `hbm` is the algorithmic bytes per second against the
+measured copy bandwidth; `launch_ms` the mean, median, min and max launch
+time), `cpu_baseline` (the fp64 oracle on a bounded sample, timed on this
+host's cores), `clocks` (nvidia-smi sampled during the timed region),
+`gpu_launches`, `exact_pass` (work items recomputed with hi + lo weights).
 
 `--impl reference` times the reference arm, which for this operator is the
 fp64 CPU oracle, on bounded samples of the same workload.
