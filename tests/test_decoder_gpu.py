@@ -120,6 +120,17 @@ def test_decoder_llama3_8b_dims_aligned():
     _check(x, w, y, m["Hq"], m["Hkv"], m["D"], "llama3-8b dims, B=2 S=256")
 
 
+def test_decoder_llama3_70b_dims():
+    """The full LLaMA3-70B layer dimensions (K = 8192 in every projection but
+    the down projection's 28672; a 57344-wide gate/up GEMM) on one short
+    ragged sequence."""
+    m = DECODER_MODELS["llama3-70b"]
+    x, w, y = _run(1, 72, m["hidden"], m["Hq"], m["Hkv"], m["D"], m["inter"], seed=73)
+    _check(x, w, y, m["Hq"], m["Hkv"], m["D"], "llama3-70b dims, S=72")
+    del x, w, y
+    torch.cuda.empty_cache()
+
+
 def test_decoder_in_place_and_deterministic():
     B, S, hidden, Hq, Hkv, D, inter = 2, 256, 256, 4, 2, 128, 512
     x, w, y = _run(B, S, hidden, Hq, Hkv, D, inter, seed=71)

@@ -335,7 +335,8 @@ def test_constant_v():
 @pytest.mark.parametrize("B,Hq,Hkv,S,D,pinned", [(1, 8, 2, 512, 128, True),
                                                  (11, 4, 2, 384, 128, True),
                                                  (3, 1, 1, 77, 64, True),
-                                                 (5, 2, 1, 200, 128, False)])
+                                                 (5, 2, 1, 200, 128, False),
+                                                 (3, 4, 2, 300, 256, True)])
 def test_host_entry_matches_device_entry(B, Hq, Hkv, S, D, pinned):
     """The host-buffer entry (a pipeline over up to 16 batch chunks on the
     library's own streams) gives the device entry's bytes, including chunks

@@ -63,6 +63,8 @@ def test_noalloc_matches_attn_fwd_two_calls(causal):
     cases.append((q2, k2, _large_v_like(v, 43), True))        # every item exact
     q3, k3, v3 = make_qkv(1, 8, 2, 329, 64, seed=44, device="cuda")
     cases.append((q3, k3, v3, False))                         # D = 64, ragged last block
+    q4, k4, v4 = make_qkv(1, 4, 2, 300, 256, seed=45, device="cuda")
+    cases.append((q4, k4, v4, False))                         # D = 256, ragged last block
     for call in range(2):  # two calls in a row: the shared array must not carry state over
         for q_, k_, v_, all_exact in cases:
             o_ref, lse_ref = attn.attn_fwd(q_, k_, v_, causal)
