@@ -26,6 +26,7 @@ def _setup():
 SMALL = [
     (1, 1, 1, 128), (1, 2, 1, 256), (1, 4, 2, 384), (2, 8, 2, 512), (1, 8, 8, 256),
     (3, 6, 3, 640),
+    (2, 32, 1, 300),  # multi-query: one kv head for 32 query heads, ragged S
 ]
 
 
@@ -593,7 +594,7 @@ def test_fma_pipe_exp2_error_bound():
 # tail, logits of standard deviation 1 and 16, one-tile and two-tile items.
 VARIANT_CASES = [(2, 4, 2, 383, 128, 1.0), (1, 8, 2, 512, 128, 4.0), (2, 4, 2, 329, 64, 1.0),
                  (1, 4, 2, 640, 64, 4.0), (1, 64, 8, 700, 128, 1.0), (2, 48, 8, 520, 128, 4.0),
-                 (1, 96, 8, 384, 64, 1.0)]
+                 (1, 96, 8, 384, 64, 1.0), (2, 32, 1, 300, 128, 1.0)]
 
 
 def _variant_check(q, k, v, causal, variant, what):
