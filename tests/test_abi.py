@@ -56,6 +56,10 @@ def test_validation_before_launch(lib):
     assert call(lib, q=None) == NULL
     assert call(lib, lse=None) == NULL
     assert call(lib, B=0) == SHAPE
+    assert call(lib, S=0) == SHAPE            # empty sequence
+    assert call(lib, Hkv=0) == SHAPE
+    assert call(lib, B=-1) == SHAPE
+    assert call(lib, S=-128) == SHAPE
     assert call(lib, Hkv=3) == SHAPE          # Hq % Hkv != 0
     assert call(lib, Hq=0) == SHAPE
     assert call(lib, D=96) == UNSUP
